@@ -7,7 +7,8 @@ comparison methods share one round-to-nearest quantizer with QuantMLA. The
 pages give no formula; the plainest reading, used here:
 
   for one token's channel group x[0..g) and b bits, qmax = 2^b - 1:
-    mn = min(x), mx = max(x)                    (exact on the bf16 inputs)
+    mn = min(x) + 0, mx = max(x)                (exact on the bf16 inputs; +0
+                                                 makes a -0.0 minimum +0.0)
     s  = fp16( fp32( fp32(mx - mn) / qmax ) )   (IEEE fp32 ops, then RN to fp16)
     z  = fp16( mn )
     u  = 0                                       if s == 0
@@ -48,7 +49,10 @@ def quantize_groups(x, bits: int, group: int):
     if d % group:
         raise ValueError("channel count must be a multiple of the group size")
     xg = x.reshape(n, d // group, group)
-    mn = xg.min(axis=-1)
+    # adding +0 turns a minimum of -0.0 into +0.0, so the zero-point of a
+    # group whose minimum is a signed zero does not depend on which zero a
+    # min-reduction happens to return
+    mn = np.add(xg.min(axis=-1), np.float32(0), dtype=np.float32)
     mx = xg.max(axis=-1)
     qmax = np.float32(qmax_of(bits))
     rng_ = np.subtract(mx, mn, dtype=np.float32)

@@ -64,7 +64,7 @@ def _brute_quantize(x, bits, group):
     for i in range(n):
         for g in range(d // group):
             vals = [f32(x[i, g * group + j]) for j in range(group)]
-            lo, hi = min(vals), max(vals)
+            lo, hi = f32(min(vals) + f32(0)), max(vals)
             s = np.float16(f32(f32(hi - lo) / f32(qmax)))
             z = np.float16(lo)
             ss[i, g], zz[i, g] = s, z
@@ -119,6 +119,15 @@ def test_roundtrip_error_bound(bits, group):
     am = xg.argmin(-1)
     ug = u.reshape(n, d // group, group)
     assert np.all(np.take_along_axis(ug, am[..., None], -1) == 0)
+
+
+def test_signed_zero_minimum_gives_positive_zero_point():
+    x = np.zeros((2, 64), dtype=np.float32)
+    x[0, 3] = -0.0
+    x[1, :] = -0.0
+    x[1, 7] = 0.5
+    _, _, z = quant.quantize_groups(x, 4, 64)
+    assert np.all(z.view(np.uint16) == 0)
 
 
 def test_constant_group_decodes_exactly():
