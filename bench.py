@@ -1,0 +1,454 @@
+"""Benchmark of the low-bit MLA decode step on B200.
+
+One step = the whole hot path over one batch: quantize + pack + paged write of
+the step's new tokens (mla_qcache_append), then the decode over the quantized
+cache (mla_qdecode: split-KV decode kernel + combine). The BF16 comparison
+decode (mla_decode_bf16) is timed as a separate leg on the same shapes.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3]
+  python bench.py --impl reference ...    # the CPU oracle, timed on host cores
+
+Prints one JSON line on rank 0. Inputs are synthetic (seeded; see
+bit_mla_kv_qdecode_b200/synth.py). L2 hygiene: every step reads a different
+copy of the cache and queries, and the copies together exceed 3x the L2 size.
+Multi-GPU runs (torchrun) are weak-scaling replicas: each rank decodes its own
+batch of the same shape, with no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KV tokens attended/sec·head-batch (head-tokens/s) and achieved HBM GB/s, 1 GPU"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_stats(w, lens):
+    """Head-tokens, KV tokens, algorithmic bytes and flops of one decode."""
+    s_q, H = w.s_q, w.H
+    vis = np.stack([np.maximum(lens.astype(np.int64) - s_q + 1 + i, 0) for i in range(s_q)], axis=1)
+    head_tokens = int(vis.sum()) * H
+    kv_tokens = int(lens.astype(np.int64).sum())
+    bpt = (512 * w.bits_c // 8 + (512 // w.group_c) * 4 + 64 * w.bits_r // 8 + (64 // w.group_r) * 4)
+    q_bytes = w.B * s_q * H * 576 * 2
+    o_bytes = w.B * s_q * H * 512 * 2
+    alg_bytes = kv_tokens * bpt + q_bytes + o_bytes
+    alg_bytes_bf16 = kv_tokens * 1152 + q_bytes + o_bytes
+    flops = 2 * head_tokens * (576 + 512)
+    return dict(head_tokens=head_tokens, kv_tokens=kv_tokens, bytes_per_token=bpt, alg_bytes=alg_bytes,
+                alg_bytes_bf16=alg_bytes_bf16, flops=flops, q_bytes=q_bytes, o_bytes=o_bytes)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples over a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_reference(args, w):
+    """The CPU oracle as it stands, timed on this host's cores on a bounded sample."""
+    from bit_mla_kv_qdecode_b200 import synth
+    from oracle import attention, layout
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    lens = synth.seq_lens(w)
+    table, num_pages = synth.block_table(w, lens)
+    desc = layout.Desc(bits_c=w.bits_c, group_c=w.group_c, bits_r=w.bits_r, group_r=w.group_r)
+    mag = synth.channel_magnitudes(w)
+    qc_bits, qr_bits = synth.queries_bf16(w)
+    qc, qr = synth.bf16_bits_to_f32(qc_bits), synth.bf16_bits_to_f32(qr_bits)
+    hist = np.maximum(lens - w.n_new, 0)
+    # sample: the first requests whose history fits a ~1.5 s packing budget per step
+    budget_tokens = 300_000
+    sample, tot = [], 0
+    for b in range(w.B):
+        if sample and tot + int(lens[b]) > budget_tokens:
+            break
+        sample.append(b)
+        tot += int(lens[b])
+    pool = np.zeros((num_pages, desc.page_bytes), dtype=np.uint8)
+    new_tok = {}
+    for b in sample:
+        x = synth.bf16_bits_to_f32(synth.cache_tokens_bf16(w, b, int(lens[b]), mag))
+        layout.append(desc, pool, table[b:b + 1], [0], x[None, :hist[b], :512], x[None, :hist[b], 512:])
+        new_tok[b] = x[hist[b]:]
+    sub = np.array(sample)
+    st = workload_stats(w.scaled(B=len(sample)), lens[sub])
+
+    def step():
+        for b in sample:
+            layout.append(desc, pool, table[b:b + 1], [hist[b]], new_tok[b][None, :, :512], new_tok[b][None, :, 512:])
+        attention.qdecode(desc, pool, table, lens, qc, qr, w.scale, requests=sample)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    cores = _blas_threads()
+    val = st["head_tokens"] / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "head-tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, args.gpus, extra={"sample_requests": len(sample)}),
+        "cpu_baseline": {"value": val, "unit": "head-tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(sample)} of {w.B} requests (all heads), append + decode per step"},
+        "e2e": {"value": val, "unit": "head-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def _config(w, n_gpus, extra=None):
+    c = {"workload": f"{w.name}: B={w.B} H={w.H} s_q={w.s_q} T={w.t_lo}"
+                     + (f"..{w.t_hi}" if w.t_hi != w.t_lo else "")
+                     + f" INT{w.bits_c} g{w.group_c} content / INT{w.bits_r} g{w.group_r} rope,"
+                     + (" paged 64-token pages" if w.paged else " contiguous"),
+         "B": w.B, "H": w.H, "s_q": w.s_q, "d_c": 512, "d_r": 64, "page": 64,
+         "n_new_per_step": w.n_new, "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "1 GPU",
+         "l2": "rotated cache+query copies > 3x L2"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def cpu_baseline_leg(w, seconds=12.0):
+    """The oracle timed on a bounded sample (rank 0, N=1 only)."""
+    from bit_mla_kv_qdecode_b200 import synth
+    from oracle import attention, quant
+    lens = synth.seq_lens(w)
+    mag = synth.channel_magnitudes(w)
+    qc_bits, qr_bits = synth.queries_bf16(w)
+    qc, qr = synth.bf16_bits_to_f32(qc_bits), synth.bf16_bits_to_f32(qr_bits)
+    head_tokens, done = 0, 0
+    t_spent = 0.0
+    for b in range(w.B):
+        x = synth.bf16_bits_to_f32(synth.cache_tokens_bf16(w, b, int(lens[b]), mag))
+        t0 = time.perf_counter()
+        u, s, z = quant.quantize_groups(x[:, :512], w.bits_c, w.group_c)
+        C = quant.dequantize_groups(u, s, z, w.group_c)
+        u, s, z = quant.quantize_groups(x[:, 512:], w.bits_r, w.group_r)
+        R = quant.dequantize_groups(u, s, z, w.group_r)
+        rq_c, rq_r, L = attention.request_rows(qc[b], qr[b], int(lens[b]))
+        attention.attend(rq_c, rq_r, C, R, w.scale, L)
+        t_spent += time.perf_counter() - t0
+        head_tokens += int(L.sum())
+        done += 1
+        if t_spent >= seconds:
+            break
+    return {"value": head_tokens / t_spent, "unit": "head-tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {w.B} requests, all heads: quantize+dequantize their cache and attend "
+                      f"(float64), {t_spent:.1f} s"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="dsv3")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from bit_mla_kv_qdecode_b200 import synth
+    w = synth.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    from bit_mla_kv_qdecode_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # ---- inputs (synthetic, seeded), resident in HBM ----
+    lens = synth.seq_lens(w)
+    table, num_pages = synth.block_table(w, lens)
+    mag = synth.channel_magnitudes(w)
+    hist = np.maximum(lens - w.n_new, 0).astype(np.int32)
+    desc = api.make_desc(w.bits_c, w.group_c, w.bits_r, w.group_r, num_pages=num_pages)
+    page_bytes = api.mla_qcache_page_bytes(desc)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    pool_bytes = num_pages * page_bytes
+    R = max(3, math.ceil(3 * l2 / pool_bytes))
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    table_t = torch.from_numpy(table).to(dev)
+    hist_t = torch.from_numpy(hist).to(dev)
+    lens_t = torch.from_numpy(lens).to(dev)
+    pool0 = api.new_qcache_pool(desc, device=dev)
+    want_bf16 = (not args.no_bf16) and num_pages * 64 * 1152 * 3 < 60e9
+    pool_b0 = api.new_bf16_pool(num_pages, device=dev) if want_bf16 else None
+    new_c = np.zeros((w.B, w.n_new, 512), dtype=np.uint16)
+    new_r = np.zeros((w.B, w.n_new, 64), dtype=np.uint16)
+    for b in range(w.B):
+        toks = synth.cache_tokens_bf16(w, b, int(lens[b]), mag)
+        for t0 in range(0, int(lens[b]), 16384):
+            part = toks[t0:t0 + 16384]
+            lb = torch.tensor([t0], dtype=torch.int32, device=dev)
+            c, r = to_dev(part[None, :, :512]), to_dev(part[None, :, 512:])
+            api.mla_qcache_append(desc, pool0, table_t[b:b + 1], lb, c, r)
+            if pool_b0 is not None:
+                api.mla_bf16cache_append(pool_b0, table_t[b:b + 1], lb, c, r)
+        new_c[b], new_r[b] = toks[hist[b]:, :512], toks[hist[b]:, 512:]
+    qc_bits, qr_bits = synth.queries_bf16(w)
+    pools = [pool0] + [pool0.clone() for _ in range(R - 1)]
+    qcs = [to_dev(qc_bits) for _ in range(R)]
+    qrs = [to_dev(qr_bits) for _ in range(R)]
+    newc_t, newr_t = to_dev(new_c), to_dev(new_r)
+    out = torch.empty((w.B, w.s_q, w.H, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.s_q, w.H), dtype=torch.float32, device=dev)
+    max_len = int(lens.max())
+    n_split = api.mla_decode_num_splits(w.B, w.s_q, w.H, max_len, w.num_splits)
+    ws_bytes = api.mla_decode_workspace_bytes(w.B, w.s_q, w.H, max_len, w.num_splits)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    assert api.mla_get_device_status() == 0
+
+    def step(k, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.mla_qcache_append(desc, pools[k], table_t, hist_t, newc_t, newr_t, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        api.mla_qdecode(desc, pools[k], table_t, lens_t, max_len, qcs[k], qrs[k], w.scale, out=out, lse=lse,
+                        num_splits=w.num_splits, workspace=ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(i % R)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i % R, evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+        dist.barrier()
+    ms_step = ms_total / args.steps
+    ms_append = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
+    ms_decode = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(args.steps))
+    assert api.mla_get_device_status() == 0
+
+    st = workload_stats(w, lens)
+    value = st["head_tokens"] * world / (ms_step * 1e-3)
+    peaks, peak_src = load_peaks()
+    flop_rate = st["flops"] / (ms_decode * 1e-3) / 1e12
+    gbs = st["alg_bytes"] / (ms_decode * 1e-3) / 1e9
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    tensor_bound = st["flops"] / st["alg_bytes"] > ridge
+    if tensor_bound:
+        roof = {"bound": "tensor", "achieved": flop_rate, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": flop_rate / peaks["bf16_tflops_sustained"], "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
+    roof["kernel"] = "mla_qdecode (decode kernel + split-KV combine, one C-ABI call)"
+    roof["per_launch_ms"] = ms_decode
+    roof["algorithmic"] = {"flops": st["flops"], "bytes": st["alg_bytes"]}
+
+    # ---- BF16 comparison decode (separate leg, same shapes) ----
+    bf16_leg = None
+    if pool_b0 is not None:
+        Rb = max(3, math.ceil(3 * l2 / (num_pages * 64 * 1152)))
+        pools_b = [pool_b0] + [pool_b0.clone() for _ in range(Rb - 1)]
+        for i in range(args.warmup):
+            api.mla_decode_bf16(pools_b[i % Rb], table_t, lens_t, max_len, qcs[i % R], qrs[i % R], w.scale,
+                                out=out, lse=lse, num_splits=w.num_splits, workspace=ws, stream=stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            api.mla_decode_bf16(pools_b[i % Rb], table_t, lens_t, max_len, qcs[i % R], qrs[i % R], w.scale,
+                                out=out, lse=lse, num_splits=w.num_splits, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_b = e0.elapsed_time(e1) / args.steps
+        bf16_leg = {"ms_per_decode": ms_b, "head_tokens_per_s": st["head_tokens"] / (ms_b * 1e-3),
+                    "alg_gbs": st["alg_bytes_bf16"] / (ms_b * 1e-3) / 1e9,
+                    "qdecode_speedup": ms_b / ms_decode}
+        del pools_b
+
+    # ---- end to end through the C ABI with host buffers ----
+    h_qc = torch.from_numpy(qc_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_qr = torch.from_numpy(qr_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_nc = torch.from_numpy(new_c.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_nr = torch.from_numpy(new_r.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    d_nc, d_nr = torch.empty_like(newc_t), torch.empty_like(newr_t)
+
+    def e2e_step(k):
+        qcs[k].copy_(h_qc, non_blocking=True)
+        qrs[k].copy_(h_qr, non_blocking=True)
+        d_nc.copy_(h_nc, non_blocking=True)
+        d_nr.copy_(h_nr, non_blocking=True)
+        api.mla_qcache_append(desc, pools[k], table_t, hist_t, d_nc, d_nr, stream=stream)
+        api.mla_qdecode(desc, pools[k], table_t, lens_t, max_len, qcs[k], qrs[k], w.scale, out=out, lse=lse,
+                        num_splits=w.num_splits, workspace=ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i % R)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i % R)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    h2d = (h_qc.numel() + h_qr.numel() + h_nc.numel() + h_nr.numel()) * 2
+    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+
+    launches_per_step = 2 + (1 if n_split > 1 else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": _config(w, world, extra={"num_splits": n_split, "pool_copies": R, "pool_mb": pool_bytes / 1e6}),
+        "kv_tokens_per_s": st["kv_tokens"] * world / (ms_step * 1e-3),
+        "hbm": {"achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+                "note": "algorithmic bytes of one decode / decode-call time"},
+        "legs_ms": {"append": ms_append, "decode": ms_decode},
+        "roofline": roof,
+        "e2e": {"value": st["head_tokens"] * world / (ms_e2e * 1e-3), "unit": "head-tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "bf16_decode": bf16_leg,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_leg(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,313 @@
+// C ABI of the low-bit MLA decode library: argument validation, split
+// planning, dispatch to the kernels, and the per-device status word.
+// Declarations and the contract of every entry point: include/mla_qcache.h.
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "mla_common.cuh"
+#include "mla_internal.h"
+
+namespace {
+
+// First error recorded by any kernel on this device since the last read.
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int* g_status_ptr[kMaxDevices] = {};
+
+// Device address of g_device_status on the current device (looked up once per
+// device; cudaGetSymbolAddress needs that device current).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t n, size_t a) { return (n + a - 1) / a * a; }
+
+bool supported_bits(int b) { return b == 2 || b == 4; }
+bool supported_group(int g) { return g == 32 || g == 64; }
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // clear a sticky "no device" from the query
+    return 148;          // B200
+  }
+  return n;
+}
+
+struct SplitPlan {
+  int n_split;
+  int chunk_pages;
+};
+
+// Split each request's pages into n page-aligned chunks. An explicit request
+// is honoured (capped at the page count). The automatic choice aims at about
+// two waves of 128-row work units over the SMs, and never cuts a request into
+// chunks shorter than 4 pages.
+SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
+  const int pages = std::max(1, (max_seq_len + mla::kPage - 1) / mla::kPage);
+  int n;
+  if (requested > 0) {
+    n = std::min(requested, pages);
+  } else {
+    const long units = static_cast<long>(std::max(B, 1)) * ((static_cast<long>(s_q) * H + 127) / 128);
+    const long slots = device_sm_count() / 2;  // one 2-CTA cluster per unit
+    long want = (2 * slots + units - 1) / units;
+    want = std::min<long>(want, (pages + 3) / 4);
+    n = static_cast<int>(std::max<long>(1, want));
+  }
+  const int chunk = (pages + n - 1) / n;
+  return SplitPlan{(pages + chunk - 1) / chunk, chunk};
+}
+
+size_t workspace_for(int B, int rows, const SplitPlan& p) {
+  if (p.n_split <= 1) return 0;
+  const size_t parts = static_cast<size_t>(B) * p.n_split * rows;
+  return align_up(parts * sizeof(float), 256) + parts * mla::kDc * sizeof(float);
+}
+
+mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
+
+struct DecodeCommon {
+  const void* pool;
+  int num_pages;
+  const int32_t* block_table;
+  int max_pages_per_seq;
+  const int32_t* seq_lens;
+  int max_seq_len;
+  const void* q_c;
+  const void* q_r;
+  int B, s_q, H;
+  float scale;
+  int num_splits;
+  void* workspace;
+  size_t workspace_bytes;
+  void* out;
+  int out_dtype;
+  float* lse;
+  unsigned flags;
+  cudaStream_t stream;
+};
+
+mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_desc* desc) {
+  if (c.B < 0 || c.s_q < 1 || c.H < 1 || c.num_pages < 0 || c.max_seq_len < 0 || c.num_splits < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (c.out_dtype != 0 && c.out_dtype != 1) return MLA_ERR_INVALID_ARG;
+  if (!isfinite(c.scale)) return MLA_ERR_INVALID_ARG;
+  if (c.flags & ~(MLA_DECODE_FORCE_SIMT | MLA_DECODE_FAST_UNCOMPENSATED)) return MLA_ERR_INVALID_ARG;
+  if (c.B == 0) return MLA_OK;
+  if (c.B > 65535 || static_cast<long>(c.s_q) * c.H > (1 << 20)) return MLA_ERR_UNSUPPORTED;
+  if (!c.block_table || !c.seq_lens || !c.q_c || !c.q_r || !c.out) return MLA_ERR_INVALID_ARG;
+  if (c.num_pages > 0 && !c.pool) return MLA_ERR_INVALID_ARG;
+  if (c.max_pages_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long>(c.max_seq_len) > static_cast<long>(c.max_pages_per_seq) * mla::kPage)
+    return MLA_ERR_CAPACITY;
+  if (!aligned(c.q_c, 16) || !aligned(c.q_r, 16) || !aligned(c.out, 16) || (c.pool && !aligned(c.pool, 256)) ||
+      !aligned(c.lse, 4))
+    return MLA_ERR_INVALID_ARG;
+  const int rows = c.s_q * c.H;
+  const SplitPlan plan = plan_splits(c.B, c.s_q, c.H, c.max_seq_len, c.num_splits);
+  if (plan.n_split > 65535) return MLA_ERR_UNSUPPORTED;
+  const size_t need = workspace_for(c.B, rows, plan);
+  if (need > 0 && (!c.workspace || c.workspace_bytes < need || !aligned(c.workspace, 256)))
+    return MLA_ERR_WORKSPACE;
+
+  int* status = status_ptr();
+  if (!status) return MLA_ERR_CUDA;
+
+  mla::DecodeLaunch L{};
+  L.pool = c.pool;
+  L.quantized = quantized;
+  if (quantized) {
+    L.bits_c = desc->bits_c;
+    L.group_c = desc->group_c;
+    L.bits_r = desc->bits_r;
+    L.group_r = desc->group_r;
+  }
+  L.num_pages = c.num_pages;
+  L.table = c.block_table;
+  L.max_pages = c.max_pages_per_seq;
+  L.seq_lens = c.seq_lens;
+  L.max_seq_len = c.max_seq_len;
+  L.q_c = c.q_c;
+  L.q_r = c.q_r;
+  L.B = c.B;
+  L.s_q = c.s_q;
+  L.H = c.H;
+  L.scale = c.scale;
+  L.n_split = plan.n_split;
+  L.chunk_pages = plan.chunk_pages;
+  if (plan.n_split > 1) {
+    const size_t parts = static_cast<size_t>(c.B) * plan.n_split * rows;
+    L.lse_part = static_cast<float*>(c.workspace);
+    L.o_part = reinterpret_cast<float*>(static_cast<char*>(c.workspace) + align_up(parts * sizeof(float), 256));
+  }
+  L.out = c.out;
+  L.out_f32 = c.out_dtype;
+  L.lse = c.lse;
+  L.flags = c.flags;
+  L.status = status;
+  L.stream = c.stream;
+
+  cudaError_t e = cudaErrorNotSupported;
+  if (!(c.flags & MLA_DECODE_FORCE_SIMT)) e = mla::launch_decode_tc(L);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = mla::launch_decode_simt(L);
+  }
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (plan.n_split > 1) return from_cuda(mla::launch_combine(L));
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: shape or bit width not supported by this build";
+    case MLA_ERR_CAPACITY: return "MLA_ERR_CAPACITY: sequence does not fit its block-table row";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA call failed";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a bounded device-side wait ran out";
+  }
+  return "unknown mla_status";
+}
+
+int mla_qcache_layout_version(void) { return MLA_QCACHE_LAYOUT_VERSION; }
+
+mla_status mla_qcache_check_desc(const mla_qcache_desc* d) {
+  if (!d) return MLA_ERR_INVALID_ARG;
+  if (d->d_c <= 0 || d->d_r <= 0 || d->bits_c <= 0 || d->bits_r <= 0 || d->group_c <= 0 || d->group_r <= 0 ||
+      d->page_size <= 0 || d->num_pages < 0)
+    return MLA_ERR_INVALID_ARG;
+  if (d->d_c % d->group_c || d->d_r % d->group_r) return MLA_ERR_INVALID_ARG;
+  if (d->d_c != mla::kDc || d->d_r != mla::kDr || d->page_size != mla::kPage) return MLA_ERR_UNSUPPORTED;
+  if (!supported_bits(d->bits_c) || !supported_bits(d->bits_r) || !supported_group(d->group_c) ||
+      !supported_group(d->group_r))
+    return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+mla_status mla_qcache_segment_offsets(const mla_qcache_desc* d, size_t out[5]) {
+  if (!out) return MLA_ERR_INVALID_ARG;
+  const mla_status st = mla_qcache_check_desc(d);
+  if (st != MLA_OK) return st;
+  const size_t P = d->page_size;
+  out[0] = 0;
+  out[1] = align_up(out[0] + P * (d->d_c * d->bits_c / 8), 16);
+  out[2] = align_up(out[1] + P * (d->d_r * d->bits_r / 8), 16);
+  out[3] = align_up(out[2] + P * (d->d_c / d->group_c) * 4, 16);
+  out[4] = align_up(out[3] + P * (d->d_r / d->group_r) * 4, 16);
+  return MLA_OK;
+}
+
+size_t mla_qcache_page_bytes(const mla_qcache_desc* d) {
+  size_t off[5];
+  return mla_qcache_segment_offsets(d, off) == MLA_OK ? off[4] : 0;
+}
+
+mla_status mla_qcache_append(const mla_qcache_desc* desc, void* pool, const int32_t* block_table,
+                             int max_pages_per_seq, const int32_t* seq_lens_before, const void* c_new,
+                             const void* kr_new, int B, int n_new, mla_stream_t stream) {
+  const mla_status st = mla_qcache_check_desc(desc);
+  if (st != MLA_OK) return st;
+  if (B < 0 || n_new < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0 || n_new == 0) return MLA_OK;
+  if (!pool || !block_table || !seq_lens_before || !c_new || !kr_new || max_pages_per_seq < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(pool, 256) || !aligned(c_new, 16) || !aligned(kr_new, 16)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long>(B) * n_new > (1L << 26)) return MLA_ERR_UNSUPPORTED;
+  int* status = status_ptr();
+  if (!status) return MLA_ERR_CUDA;
+  mla::AppendLaunch L{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens_before, c_new, kr_new,
+                      B, n_new, desc->bits_c, desc->group_c, desc->bits_r, desc->group_r, status,
+                      reinterpret_cast<cudaStream_t>(stream)};
+  return from_cuda(mla::launch_qcache_append(L));
+}
+
+mla_status mla_bf16cache_append(void* pool, int num_pages, int page_size, const int32_t* block_table,
+                                int max_pages_per_seq, const int32_t* seq_lens_before, const void* c_new,
+                                const void* kr_new, int B, int n_new, mla_stream_t stream) {
+  if (page_size != mla::kPage) return page_size > 0 ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  if (B < 0 || n_new < 0 || num_pages < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0 || n_new == 0) return MLA_OK;
+  if (!pool || !block_table || !seq_lens_before || !c_new || !kr_new || max_pages_per_seq < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned(pool, 256) || !aligned(c_new, 16) || !aligned(kr_new, 16)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long>(B) * n_new > (1L << 26)) return MLA_ERR_UNSUPPORTED;
+  int* status = status_ptr();
+  if (!status) return MLA_ERR_CUDA;
+  mla::AppendLaunch L{pool, num_pages, block_table, max_pages_per_seq, seq_lens_before, c_new, kr_new,
+                      B, n_new, 0, 0, 0, 0, status, reinterpret_cast<cudaStream_t>(stream)};
+  return from_cuda(mla::launch_bf16cache_append(L));
+}
+
+int mla_decode_num_splits(int B, int s_q, int H, int max_seq_len, int num_splits) {
+  if (B < 0 || s_q < 1 || H < 1 || max_seq_len < 0 || num_splits < 0) return 0;
+  return plan_splits(B, s_q, H, max_seq_len, num_splits).n_split;
+}
+
+size_t mla_decode_workspace_bytes(int B, int s_q, int H, int max_seq_len, int num_splits) {
+  if (B <= 0 || s_q < 1 || H < 1 || max_seq_len < 0 || num_splits < 0) return 0;
+  return workspace_for(B, s_q * H, plan_splits(B, s_q, H, max_seq_len, num_splits));
+}
+
+mla_status mla_qdecode(const mla_qcache_desc* desc, const void* pool, const int32_t* block_table,
+                       int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, const void* q_c,
+                       const void* q_r, int B, int s_q, int H, float scale, int num_splits, void* workspace,
+                       size_t workspace_bytes, void* out, int out_dtype, float* lse, unsigned flags,
+                       mla_stream_t stream) {
+  const mla_status st = mla_qcache_check_desc(desc);
+  if (st != MLA_OK) return st;
+  DecodeCommon c{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens, max_seq_len, q_c, q_r,
+                 B, s_q, H, scale, num_splits, workspace, workspace_bytes, out, out_dtype, lse, flags,
+                 reinterpret_cast<cudaStream_t>(stream)};
+  return run_decode(c, true, desc);
+}
+
+mla_status mla_decode_bf16(const void* pool, int num_pages, int page_size, const int32_t* block_table,
+                           int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len, const void* q_c,
+                           const void* q_r, int B, int s_q, int H, float scale, int num_splits, void* workspace,
+                           size_t workspace_bytes, void* out, int out_dtype, float* lse, unsigned flags,
+                           mla_stream_t stream) {
+  if (page_size != mla::kPage) return page_size > 0 ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  DecodeCommon c{pool, num_pages, block_table, max_pages_per_seq, seq_lens, max_seq_len, q_c, q_r,
+                 B, s_q, H, scale, num_splits, workspace, workspace_bytes, out, out_dtype, lse, flags,
+                 reinterpret_cast<cudaStream_t>(stream)};
+  return run_decode(c, false, nullptr);
+}
+
+mla_status mla_get_device_status(int* status, mla_stream_t stream) {
+  if (!status) return MLA_ERR_INVALID_ARG;
+  *status = MLA_OK;
+  if (!status_ptr()) return MLA_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  *status = v;
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+struct AppendLaunch {
+  void* pool;
+  int num_pages;
+  const int32_t* table;
+  int max_pages;
+  const int32_t* lens_before;
+  const void* c_new;
+  const void* kr_new;
+  int B, n_new;
+  int bits_c, group_c, bits_r, group_r;
+  int* status;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_qcache_append(const AppendLaunch& L);
+cudaError_t launch_bf16cache_append(const AppendLaunch& L);
+
+// One decode call, after validation and split planning.
+struct DecodeLaunch {
+  const void* pool;
+  bool quantized;
+  int bits_c, group_c, bits_r, group_r;
+  int num_pages;
+  const int32_t* table;
+  int max_pages;
+  const int32_t* seq_lens;
+  int max_seq_len;
+  const void* q_c;
+  const void* q_r;
+  int B, s_q, H;
+  float scale;
+  int n_split, chunk_pages;
+  float* o_part;   // workspace (n_split > 1)
+  float* lse_part;
+  void* out;
+  int out_f32;
+  float* lse;
+  unsigned flags;
+  int* status;
+  cudaStream_t stream;
+};
+
+struct DecodeArgs;
+DecodeArgs make_decode_args(const DecodeLaunch& L);
+
+cudaError_t launch_decode_simt(const DecodeLaunch& L);
+cudaError_t launch_combine(const DecodeLaunch& L);
+// Returns cudaErrorNotSupported when the tensor-core kernel has no variant for
+// the shape; the caller then uses the SIMT kernel.
+cudaError_t launch_decode_tc(const DecodeLaunch& L);
+
+}  // namespace mla

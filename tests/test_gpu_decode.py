@@ -1,0 +1,150 @@
+"""GPU parity of the decode path against the float64 oracle.
+
+Bar (fp32 output): max |o - o_ref| <= 2e-3 * RMS(o_ref) over the checked
+rows; bf16 output adds half a bf16 ulp of the value. lse within 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bit_mla_kv_qdecode_b200 import MLA_DECODE_FORCE_SIMT, api, synth
+from tests import mla_cases as mc
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [0, MLA_DECODE_FORCE_SIMT]
+
+
+def run_decode(case, pool, table_t, flags=0, num_splits=0, out_dtype=torch.float32, quantized=True,
+               lens=None):
+    w = case.w
+    qc, qr = mc.device_queries(case)
+    lens_t = torch.from_numpy(case.lens if lens is None else lens).cuda()
+    lse = torch.empty((w.B, w.s_q, w.H), dtype=torch.float32, device="cuda")
+    if quantized:
+        out, _ = api.mla_qdecode(case.desc, pool, table_t, lens_t, case.max_seq_len, qc, qr, w.scale,
+                                 out_dtype=out_dtype, lse=lse, num_splits=num_splits, flags=flags)
+    else:
+        out, _ = api.mla_decode_bf16(pool, table_t, lens_t, case.max_seq_len, qc, qr, w.scale,
+                                     out_dtype=out_dtype, lse=lse, num_splits=num_splits, flags=flags)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def check(case, out, lse, requests, quantized=True, bf16_out=False):
+    ref = mc.oracle_decode(case, requests, quantized)
+    err, lerr = mc.parity(out, lse, ref, bf16_out=bf16_out)
+    assert err <= mc.RTOL_RMS, f"max err {err:.3e} x RMS"
+    assert lerr <= mc.LSE_ATOL, f"lse err {lerr:.3e}"
+    return err
+
+
+SMALL = [
+    # (bits_c, group_c, bits_r, group_r, H, s_q, lens)
+    (4, 64, 4, 64, 128, 1, [1, 63, 64, 65, 200, 1000]),
+    (2, 32, 4, 64, 128, 1, [130, 1, 777]),
+    (2, 32, 4, 64, 128, 2, [2, 65, 300, 1024]),
+    (4, 64, 4, 64, 16, 1, [1024, 5]),
+    (4, 32, 2, 64, 32, 2, [100, 129]),
+    (2, 64, 2, 32, 64, 1, [640, 64]),
+    (4, 64, 4, 64, 8, 3, [3, 70]),
+]
+
+
+@pytest.mark.parametrize("flags", KERNELS)
+@pytest.mark.parametrize("spec", SMALL)
+@pytest.mark.parametrize("num_splits", [1, 3, 0])
+def test_decode_small_cases(spec, num_splits, flags):
+    bc, gc, br, gr, H, s_q, lens = spec
+    w = synth.workload(2).scaled(B=len(lens), H=H, s_q=s_q, bits_c=bc, group_c=gc, bits_r=br, group_r=gr)
+    case = mc.make_case(w, lens=lens)
+    pool, table_t = mc.fill_pool(case)
+    out, lse = run_decode(case, pool, table_t, flags=flags, num_splits=num_splits)
+    assert api.mla_get_device_status() == 0
+    check(case, out, lse, range(w.B))
+
+
+@pytest.mark.parametrize("flags", KERNELS)
+def test_decode_bf16_output(flags):
+    w = synth.workload(1).scaled(B=3)
+    case = mc.make_case(w, lens=[64, 500, 1])
+    pool, table_t = mc.fill_pool(case)
+    out, lse = run_decode(case, pool, table_t, flags=flags, out_dtype=torch.bfloat16)
+    assert out.dtype == torch.bfloat16
+    check(case, out, lse, range(w.B), bf16_out=True)
+
+
+@pytest.mark.parametrize("flags", KERNELS)
+@pytest.mark.parametrize("num_splits", [1, 4])
+def test_bf16_cache_decode(flags, num_splits):
+    w = synth.workload(3).scaled(B=3, s_q=2)
+    case = mc.make_case(w, lens=[65, 1000, 2])
+    pool, table_t = mc.fill_pool(case, quantized=False)
+    out, lse = run_decode(case, pool, table_t, flags=flags, num_splits=num_splits, quantized=False)
+    check(case, out, lse, range(w.B), quantized=False)
+
+
+def test_empty_request_and_length_errors():
+    w = synth.workload(1).scaled(B=3)
+    case = mc.make_case(w, lens=[0, 70, 0])
+    pool, table_t = mc.fill_pool(case)
+    for splits in (1, 2):
+        out, lse = run_decode(case, pool, table_t, num_splits=splits)
+        o = out.cpu().numpy()
+        assert np.all(o[0] == 0) and np.all(o[2] == 0)
+        assert np.all(np.isneginf(lse.cpu().numpy()[[0, 2]]))
+        check(case, out, lse, [1])
+    assert api.mla_get_device_status() == 0
+    # a device length above max_seq_len is clamped and flagged, never read past
+    bad = case.lens.copy()
+    bad[1] = 10_000
+    run_decode(case, pool, table_t, lens=bad)
+    assert api.mla_get_device_status() == api._lib.MLA_ERR_INVALID_ARG
+
+
+def test_determinism_and_paging_invariance():
+    w = synth.workload(2).scaled(B=3, H=128)
+    lens = [333, 1024, 65]
+    paged = mc.make_case(w, lens=lens)
+    flat = mc.make_case(w.scaled(paged=False), lens=lens)
+    assert not np.array_equal(paged.table, flat.table)
+    outs = []
+    for case in (paged, flat):
+        pool, table_t = mc.fill_pool(case)
+        outs.append(run_decode(case, pool, table_t, num_splits=2))
+    again = run_decode(paged, *mc.fill_pool(paged), num_splits=2)
+    for a, b in ((outs[0], again), (outs[0], outs[1])):
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_split_counts_agree():
+    w = synth.workload(3).scaled(B=1, t_lo=8192, t_hi=8192)
+    case = mc.make_case(w)
+    pool, table_t = mc.fill_pool(case)
+    ref = mc.oracle_decode(case, [0])
+    errs = []
+    for splits in (1, 7, 32, 128):
+        out, lse = run_decode(case, pool, table_t, num_splits=splits)
+        errs.append(mc.parity(out, lse, ref)[0])
+    assert max(errs) <= mc.RTOL_RMS, errs
+
+
+# Full-size workloads in the launch configuration the benchmark times (auto
+# split plan, bf16 output), oracle on a sample of requests.
+FULL = {0: [0], 1: [0, 31], 2: [5, 40], 3: [2], 4: [0, 77], 5: [3]}
+
+
+@pytest.mark.parametrize("idx", sorted(FULL))
+def test_full_size_workloads(idx):
+    w = synth.workload(idx)
+    case = mc.make_case(w)
+    pool, table_t = mc.fill_pool(case)
+    out, lse = run_decode(case, pool, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16)
+    assert api.mla_get_device_status() == 0
+    check(case, out, lse, FULL[idx], bf16_out=True)
+    if w.bf16_compare:
+        del pool
+        pool_b, _ = mc.fill_pool(case, quantized=False)
+        out, lse = run_decode(case, pool_b, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16,
+                              quantized=False)
+        check(case, out, lse, FULL[idx], quantized=False, bf16_out=True)
