@@ -1,9 +1,711 @@
-// Tensor-core (tcgen05 / TMEM) decode kernel for sm_100a.
+// Tensor-core decode for sm_100a: tcgen05 MMAs with TMEM accumulators over a
+// TMA-staged, low-bit quantized latent cache.
+//
+// Computation (absorbed MQA form of MLA decode, Group-Query Latent Attention
+// abstract, thelatestinai.com/papers/2607.27269; unpack + dequant inside the
+// attention, QuantMLA abstract, arxivdaily.com/papers/2609.36760):
+//   S[r,t] = (q_c[r] . c_hat[t] + q_r[r] . kr_hat[t]) * scale
+//   O[r,:] = sum_t softmax_t(S[r,:]) c_hat[t]
+// for 128 query rows r (heads x queries of one request) at a time.
+//
+// Work unit and cluster split. A unit is (request, key split, 128-row tile).
+// It runs on a cluster of two CTAs; CTA k owns latent channels
+// [256k, 256k+256) and RoPE channels [32k, 32k+32). Each CTA dequantizes only
+// its half of every token, computes a partial score over its 288 channels,
+// and the two partial scores are exchanged through distributed shared memory
+// and added (fp32 addition commutes, so both CTAs hold bit-identical scores
+// and take identical softmax decisions). Each CTA then accumulates its own
+// 256-wide half of the output: O_half = 128 x 256 fp32 fits TMEM beside the
+// score buffers and the query operand.
+//
+// Precision. The dequantized values u*s+z are split into bf16 hi + bf16 lo
+// (16 significant bits together), and so are the softmax weights. Scores use
+// Q*C_hi + Q*C_lo (Q is exact in bf16); the output uses P_hi*C_hi + P_lo*C_hi
+// + P_hi*C_lo. All accumulation is fp32 in TMEM. This keeps the output within
+// 2e-3 of its RMS of the exact float64 result; single bf16 operands would not.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: packed codes + metadata of 32-token chunks
+//   warp 1      TMEM owner and the single MMA-issuing thread
+//   warps 2-5   unpack + dequantize into bf16 hi/lo operand tiles
+//   warps 8-11  one thread per row: score exchange, online softmax, P tiles,
+//               output rescaling in TMEM, epilogue
+// Every wait is bounded; a timeout sets MLA_ERR_TIMEOUT and the unit drains
+// and exits without touching memory it does not own.
+#include <cuda.h>
+#include <math_constants.h>
+
+#include <mutex>
+
 #include "mla_common.cuh"
 #include "mla_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
+namespace tc {
 
-cudaError_t launch_decode_tc(const DecodeLaunch&) { return cudaErrorNotSupported; }
+constexpr int kThreads = 384;
+constexpr int kChunk = 32;            // tokens per pipeline step
+constexpr int kRows = 128;            // query rows per unit (MMA M)
+constexpr int kHalfC = 256;           // content channels per CTA
+constexpr int kHalfR = 32;            // rope channels per CTA
+constexpr int kKChunks = (kHalfC + kHalfR) / 8;  // 36 eight-channel chunks per token
+constexpr int kNC = 3;                // operand-tile stages
+constexpr int kNS = 4;                // TMA code stages
+constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (weights stay <= 2^8)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr unsigned kFull = 0xffffffffu;
+
+// TMEM columns
+constexpr uint32_t kTmemO = 0;        // 256 fp32 columns: this CTA's half of O
+constexpr uint32_t kTmemS = 256;      // two 32-column score buffers
+constexpr uint32_t kTmemQ = 320;      // 144 columns: Q (288 bf16 per row)
+constexpr uint32_t kTmemCols = 512;
+
+// Shared memory layout (bytes)
+constexpr int kCTile = kKChunks * 4 * 128;         // one bf16 operand tile: 36 chunks x 4 token groups x 128 B
+constexpr int kCStage = 2 * kCTile;                // hi + lo
+constexpr int kPTile = (kRows / 8) * 4 * 128;      // 8 KB: 16 row groups x 4 token groups x 128 B
+constexpr int kXRow = 36;                          // floats per row in the score-exchange buffer
+constexpr int kXBuf = kRows * kXRow * 4;
+constexpr int kCodeCC = 4096;                      // content codes half (32 tokens x <=128 B)
+constexpr int kCodeRC = 1024;                      // rope codes (32 tokens x <=32 B)
+constexpr int kCodeCM = 1024;                      // content meta half (32 tokens x <=32 B)
+constexpr int kCodeStage = 8192;                   // each sub-buffer 1024-aligned inside
+constexpr int kOffC = 0;
+constexpr int kOffP = kOffC + kNC * kCStage;
+constexpr int kOffX = kOffP + 2 * 2 * kPTile;
+constexpr int kOffCode = kOffX + 2 * kXBuf;
+constexpr int kOffBar = kOffCode + kNS * kCodeStage;
+constexpr int kNumBars = 2 * kNS + 2 * kNC + 2 + 2 + 2 + 2 + 2 + 2 + 2;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64;
+constexpr int kSmemAlloc = kSmemBytes + 1024;      // slack to align the base to 1024
+static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0, "TMA swizzle needs 1024-byte aligned stages");
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kSmemAlloc > 232448 / 2, "one CTA per SM keeps the 512-column TMEM allocation uncontended");
+
+struct TmapSet {
+  CUtensorMap cc;  // content codes [pages][64][row_c] bytes, box = half row x 32 tokens
+  CUtensorMap rc;  // rope codes    [pages][64][row_r], box = full row x 32 tokens
+  CUtensorMap cm;  // content meta  [pages][64][groups_c*4], box = half x 32 tokens
+};
+
+struct Bars {
+  uint64_t* code_full;   // [kNS] TMA -> dequant
+  uint64_t* code_empty;  // [kNS] dequant -> TMA
+  uint64_t* c_full;      // [kNC] dequant -> MMA
+  uint64_t* c_empty;     // [kNC] MMA (after PV) -> dequant
+  uint64_t* s_full;      // [2] MMA (QK) -> softmax
+  uint64_t* s_empty;     // [2] softmax read S -> MMA
+  uint64_t* p_full;      // [2] softmax P tile + O rescale -> MMA
+  uint64_t* p_empty;     // [2] MMA (PV) -> softmax
+  uint64_t* x_full;      // [2] peer wrote its partial scores into my exchange buffer
+  uint64_t* x_empty;     // [2] peer consumed what I wrote into its exchange buffer
+  uint64_t* q_full;      // [1] Q in TMEM
+  uint64_t* o_full;      // [1] all MMAs of the unit done
+};
+
+__device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
+  uint64_t* b = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  Bars r;
+  r.code_full = b;
+  r.code_empty = b + kNS;
+  r.c_full = b + 2 * kNS;
+  r.c_empty = b + 2 * kNS + kNC;
+  uint64_t* p = b + 2 * kNS + 2 * kNC;
+  r.s_full = p;
+  r.s_empty = p + 2;
+  r.p_full = p + 4;
+  r.p_empty = p + 6;
+  r.x_full = p + 8;
+  r.x_empty = p + 10;
+  r.q_full = p + 12;
+  r.o_full = p + 13;
+  return r;
+}
+
+__device__ __forceinline__ float u2f(uint32_t u) {  // exact for u < 2^23
+  return __uint_as_float(u | 0x4B000000u) - 8388608.0f;
+}
+
+// bf16 hi/lo of 8 values, packed two per 32-bit word (lower channel in the low half).
+__device__ __forceinline__ void split8(const float (&x)[8], uint4& hi, uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * k], x[2 * k + 1]);
+    const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+    const float h0 = __uint_as_float(hw << 16), h1 = __uint_as_float(hw & 0xFFFF0000u);
+    __nv_bfloat162 lb = __floats2bfloat162_rn(x[2 * k] - h0, x[2 * k + 1] - h1);
+    h[k] = hw;
+    l[k] = *reinterpret_cast<uint32_t*>(&lb);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+template <int BITS>
+__device__ __forceinline__ void dequant8(uint32_t w, float s, float z, float (&x)[8]) {
+  constexpr uint32_t mask = (1u << BITS) - 1u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x[k] = fmaf(u2f((w >> (k * BITS)) & mask), s, z);
+}
+
+__device__ __forceinline__ void fail(const DecodeArgs& a, volatile int* abort_flag) {
+  record_error(a.status, MLA_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
+template <int BITS_C, int G_C, int BITS_R, int G_R>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TmapSet tm, int row_tiles, int n_terms_qk,
+                     int n_terms_pv) {
+  using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Bars bars = carve_bars(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t crank = ptx::cluster_ctarank();
+  const uint32_t peer = crank ^ 1u;
+
+  // ---- unit ----
+  const int unit = blockIdx.x >> 1;
+  const int rt = unit % row_tiles;
+  const int split = (unit / row_tiles) % a.n_split;
+  const int b = unit / (row_tiles * a.n_split);
+  const int T = checked_len(a, b);
+  const int pages_b = (T + kPage - 1) / kPage;
+  const int p_begin = split * a.chunk_pages;
+  if (a.n_split > 1 && p_begin >= pages_b) return;  // both CTAs of the cluster leave together
+  const int t_begin = min(p_begin * kPage, T);
+  const int t_end = min(T, (p_begin + a.chunk_pages) * kPage);
+  const int n_chunks = (t_end - t_begin + kChunk - 1) / kChunk;
+  const int row0 = rt * kRows;
+
+  if (n_chunks == 0) {  // no keys: o = 0, lse = -inf (single-split plans write the output)
+    if (tid < kRows) {
+      const int row = row0 + tid;
+      if (row < a.rows) {
+        const size_t qrow = static_cast<size_t>(b) * a.rows + row;
+        for (int c = 0; c < kHalfC; ++c) {
+          const size_t off = qrow * kDc + crank * kHalfC + c;
+          if (a.n_split == 1) {
+            if (a.out_f32) static_cast<float*>(a.out)[off] = 0.0f;
+            else static_cast<__nv_bfloat16*>(a.out)[off] = __float2bfloat16_rn(0.0f);
+          } else {
+            a.o_part[((static_cast<size_t>(b) * a.n_split + split) * a.rows + row) * kDc + crank * kHalfC + c] = 0.f;
+          }
+        }
+        if (crank == 0) {
+          if (a.n_split == 1) { if (a.lse) a.lse[qrow] = -CUDART_INF_F; }
+          else a.lse_part[(static_cast<size_t>(b) * a.n_split + split) * a.rows + row] = -CUDART_INF_F;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---- setup ----
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      ptx::mbar_init(&bars.code_full[i], 1);
+      ptx::mbar_init(&bars.code_empty[i], 128);
+    }
+    for (int i = 0; i < kNC; ++i) {
+      ptx::mbar_init(&bars.c_full[i], 128);
+      ptx::mbar_init(&bars.c_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars.s_full[i], 1);
+      ptx::mbar_init(&bars.s_empty[i], 128);
+      ptx::mbar_init(&bars.p_full[i], 128);
+      ptx::mbar_init(&bars.p_empty[i], 1);
+      ptx::mbar_init(&bars.x_full[i], 128);
+      ptx::mbar_init(&bars.x_empty[i], 128);
+    }
+    ptx::mbar_init(bars.q_full, 128);
+    ptx::mbar_init(bars.o_full, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init_cluster();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tm.cc);
+    ptx::prefetch_tmap(&tm.rc);
+    ptx::prefetch_tmap(&tm.cm);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // peer barriers are initialised before any remote arrive
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      const uint32_t bytes = kChunk * (G::kRowC / 2) + kChunk * G::kRowR + kChunk * (G::kGroupsC * 2) +
+                             kChunk * G::kGroupsR * 4;
+      int issued[kNS];
+      for (int i = 0; i < kNS; ++i) issued[i] = 0;
+      for (int j = 0; j < n_chunks; ++j) {
+        const int s = j % kNS;
+        if (j >= kNS && !ptx::mbar_wait(&bars.code_empty[s], ((j - kNS) / kNS) & 1, abort_flag, kWaitLimitNs)) {
+          fail(a, abort_flag);
+          break;
+        }
+        const int t0 = t_begin + j * kChunk;
+        const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
+        uint8_t* st = smem + kOffCode + s * kCodeStage;
+        if (page >= 0) {
+          ptx::mbar_arrive_expect_tx(&bars.code_full[s], bytes);
+          const int slot0 = t0 % kPage;
+          ptx::tma_load_3d(st, &tm.cc, crank * (G::kRowC / 2), slot0, page, &bars.code_full[s]);
+          ptx::tma_load_3d(st + kCodeCC, &tm.rc, 0, slot0, page, &bars.code_full[s]);
+          ptx::tma_load_3d(st + kCodeCC + kCodeRC, &tm.cm, crank * (G::kGroupsC * 2), slot0, page,
+                           &bars.code_full[s]);
+          const uint8_t* rm = a.pool + static_cast<size_t>(page) * G::kPageBytes + G::kOffRM +
+                              static_cast<size_t>(slot0) * G::kGroupsR * 4;
+          ptx::bulk_load(st + kCodeCC + kCodeRC + kCodeCM, rm, kChunk * G::kGroupsR * 4, &bars.code_full[s]);
+        } else {
+          record_error(a.status, MLA_ERR_INVALID_ARG);
+          ptx::mbar_arrive(&bars.code_full[s]);
+        }
+        issued[s] = j + 1;
+      }
+      // drain copies still in flight before the CTA can exit
+      for (int s = 0; s < kNS; ++s)
+        if (issued[s] > 0) ptx::mbar_wait(&bars.code_full[s], ((issued[s] - 1) / kNS) & 1, nullptr, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // =========================== MMA issuer ===========================
+    if (lane == 0) {
+      const uint32_t idesc_qk = ptx::idesc_bf16_f32(kRows, kChunk, 0, 0);
+      const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, kHalfC, 0, 1);
+      const uint32_t c_base = ptx::smem_u32(smem + kOffC);
+      const uint32_t p_base = ptx::smem_u32(smem + kOffP);
+      bool ok = ptx::mbar_wait(bars.q_full, 0, abort_flag, kWaitLimitNs);
+      ptx::tc_fence_after();
+      auto issue_pv = [&](int j) -> bool {
+        const int pb = j & 1, cs = j % kNC;
+        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
+        ptx::tc_fence_after();
+        const uint32_t pt = p_base + pb * 2 * kPTile;
+        const uint32_t ct = c_base + cs * kCStage;
+        for (int term = 0; term < n_terms_pv; ++term) {
+          const uint32_t pa = pt + (term == 1 ? kPTile : 0);     // P_lo for term 1
+          const uint32_t cb = ct + (term == 2 ? kCTile : 0);     // C_lo for term 2
+#pragma unroll
+          for (int k = 0; k < kChunk / 16; ++k) {
+            const uint64_t ad = ptx::smem_desc_noswizzle(pa + k * 256, 128, 512);
+            const uint64_t bd = ptx::smem_desc_noswizzle(cb + k * 256, 128, 512);
+            ptx::mma_ss(tmem + kTmemO, ad, bd, idesc_pv, (j > 0 || term > 0 || k > 0) ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit(&bars.p_empty[pb]);
+        ptx::mma_commit(&bars.c_empty[cs]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_chunks; ++j) {
+        const int cs = j % kNC, sb = j & 1;
+        if (!ptx::mbar_wait(&bars.c_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        if (j >= 2 && !ptx::mbar_wait(&bars.s_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t ct = c_base + cs * kCStage;
+        for (int term = 0; term < n_terms_qk; ++term) {
+          const uint32_t cb = ct + term * kCTile;
+#pragma unroll 6
+          for (int k = 0; k < kKChunks / 2; ++k) {
+            const uint64_t bd = ptx::smem_desc_noswizzle(cb + k * 2 * 512, 512, 128);
+            ptx::mma_ts(tmem + kTmemS + sb * kChunk, tmem + kTmemQ + k * 8, bd, idesc_qk,
+                        (term > 0 || k > 0) ? 1u : 0u);
+          }
+        }
+        ptx::mma_commit(&bars.s_full[sb]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(n_chunks - 1);
+      if (!ok) fail(a, abort_flag);
+      ptx::mma_commit(bars.o_full);
+      // every issued MMA must finish before TMEM is released, abort or not
+      ptx::mbar_wait(bars.o_full, 0, nullptr, kWaitLimitNs);
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // =========================== dequant ===========================
+    const int dq = tid - 64;
+    const int tq = dq & 31;       // token within the chunk
+    const int qsel = dq >> 5;     // 0..3
+    for (int j = 0; j < n_chunks; ++j) {
+      const int s = j % kNS, cs = j % kNC;
+      if (!ptx::mbar_wait(&bars.code_full[s], (j / kNS) & 1, abort_flag, kWaitLimitNs)) { fail(a, abort_flag); break; }
+      if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, kWaitLimitNs)) {
+        fail(a, abort_flag);
+        break;
+      }
+      const int t0 = t_begin + j * kChunk;
+      const bool valid = (t0 + tq < t_end) && lookup_page(a.table, a.max_pages, a.num_pages, b, t0) >= 0;
+      const uint8_t* st = smem + kOffCode + s * kCodeStage;
+      uint8_t* chi = smem + kOffC + cs * kCStage;
+      uint8_t* clo = chi + kCTile;
+      // content: quads qsel and qsel+4 (32 channels each)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int q = qsel + 4 * h;
+        const uint32_t meta = *reinterpret_cast<const uint32_t*>(st + kCodeCC + kCodeRC +
+                                                                 tq * (G::kGroupsC * 2) + ((q * 32) / G_C) * 4);
+        const float sc = half_bits_to_float(meta), zc = half_bits_to_float(meta >> 16);
+        uint32_t w[4];
+        if constexpr (BITS_C == 4) {  // 16 B per quad, 128-byte swizzled rows
+          const uint4 v = *reinterpret_cast<const uint4*>(st + tq * 128 + ((q ^ (tq & 7)) * 16));
+          w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+        } else {                      // 8 B per quad, 64-byte swizzled rows
+          const uint2 v = *reinterpret_cast<const uint2*>(st + tq * 64 + ((((q >> 1) ^ ((tq >> 1) & 3)) * 16)) +
+                                                           (q & 1) * 8);
+          w[0] = v.x & 0xFFFFu; w[1] = v.x >> 16; w[2] = v.y & 0xFFFFu; w[3] = v.y >> 16;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
+          if (valid) {
+            float x[8];
+            dequant8<BITS_C>(w[i], sc, zc, x);
+            split8(x, hi, lo);
+          }
+          const int off = (4 * q + i) * 512 + tq * 16;
+          *reinterpret_cast<uint4*>(chi + off) = hi;
+          *reinterpret_cast<uint4*>(clo + off) = lo;
+        }
+      }
+      {  // rope: 8 channels (chunk qsel of this CTA's 32)
+        const uint32_t meta = *reinterpret_cast<const uint32_t*>(st + kCodeCC + kCodeRC + kCodeCM +
+                                                                 tq * G::kGroupsR * 4 + (G_R == 64 ? 0 : crank) * 4);
+        const float sr = half_bits_to_float(meta), zr = half_bits_to_float(meta >> 16);
+        const uint8_t* row = st + kCodeCC + tq * G::kRowR + crank * (G::kRowR / 2);
+        const uint32_t w = (BITS_R == 4) ? *reinterpret_cast<const uint32_t*>(row + qsel * 4)
+                                         : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + qsel * 2));
+        uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
+        if (valid) {
+          float x[8];
+          dequant8<BITS_R>(w, sr, zr, x);
+          split8(x, hi, lo);
+        }
+        const int off = (32 + qsel) * 512 + tq * 16;
+        *reinterpret_cast<uint4*>(chi + off) = hi;
+        *reinterpret_cast<uint4*>(clo + off) = lo;
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(&bars.c_full[cs]);
+      ptx::mbar_arrive(&bars.code_empty[s]);
+    }
+  } else if (warp >= 8) {
+    // =========================== softmax / epilogue ===========================
+    const int i = tid - 256;  // row within the tile == TMEM lane
+    const int row = row0 + i;
+    const bool row_ok = row < a.rows;
+    const int L = row_ok ? row_visible(T, a.s_q, a.H, row) : 0;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const size_t qrow = static_cast<size_t>(b) * a.rows + (row_ok ? row : 0);
+
+    // Q half -> TMEM columns [320, 464) (zeros for padding rows)
+    {
+      const uint4* qc = reinterpret_cast<const uint4*>(a.q_c + qrow * kDc + crank * kHalfC);
+      const uint4* qr = reinterpret_cast<const uint4*>(a.q_r + qrow * kDr + crank * kHalfR);
+#pragma unroll
+      for (int blk = 0; blk < 5; ++blk) {
+        uint32_t v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c16 = blk * 8 + k;  // 16-byte piece (8 bf16) index, 36 pieces
+          uint4 x = make_uint4(0, 0, 0, 0);
+          if (row_ok && c16 < 32) x = __ldg(qc + c16);
+          else if (row_ok && c16 < 36) x = __ldg(qr + (c16 - 32));
+          v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+        }
+        ptx::tmem_st32(lane_base + kTmemQ + blk * 32, v);
+      }
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bars.q_full);
+    }
+
+    const uint32_t xbuf_local = ptx::smem_u32(smem + kOffX);
+    const uint32_t xbuf_peer = ptx::mapa(xbuf_local, peer);
+    const uint32_t xfull_peer = ptx::mapa(ptx::smem_u32(bars.x_full), peer);
+    const uint32_t xempty_peer = ptx::mapa(ptx::smem_u32(bars.x_empty), peer);
+    float m_used = -CUDART_INF_F, l_sum = 0.0f;
+    bool o_live = false;  // O has been written by a PV MMA
+    bool ok = true;
+
+    for (int j = 0; j < n_chunks && ok; ++j) {
+      const int sb = j & 1;
+      const int t0 = t_begin + j * kChunk;
+      // wait results are made warp-uniform: the TMEM loads below are warp-collective
+      if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      uint32_t sv[32];
+      ptx::tmem_ld32(lane_base + kTmemS + sb * kChunk, sv);
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars.s_empty[sb]);
+
+      // exchange partial scores with the peer CTA
+      if (j >= 2 &&
+          !__all_sync(kFull, ptx::mbar_wait<true>(&bars.x_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      const uint32_t my_row_peer = xbuf_peer + sb * kXBuf + i * (kXRow * 4);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        ptx::st_cluster_v4(my_row_peer + k * 16, __uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1]),
+                           __uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3]));
+      ptx::mbar_arrive_remote(xfull_peer + sb * 8);
+      if (!__all_sync(kFull, ptx::mbar_wait<true>(&bars.x_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + sb * kXBuf + i * (kXRow * 4));
+      float s2[32];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 pv = xr[k];
+        s2[4 * k] = __uint_as_float(sv[4 * k]) + pv.x;
+        s2[4 * k + 1] = __uint_as_float(sv[4 * k + 1]) + pv.y;
+        s2[4 * k + 2] = __uint_as_float(sv[4 * k + 2]) + pv.z;
+        s2[4 * k + 3] = __uint_as_float(sv[4 * k + 3]) + pv.w;
+      }
+      ptx::mbar_arrive_remote(xempty_peer + sb * 8);
+
+      // mask + scale (log2 domain)
+      const bool page_ok = lookup_page(a.table, a.max_pages, a.num_pages, b, t0) >= 0;
+      const int lim = page_ok ? min(L, t_end) - t0 : 0;
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        s2[k] = (k < lim) ? s2[k] * a.scale_log2 : -CUDART_INF_F;
+        mx = fmaxf(mx, s2[k]);
+      }
+      float alpha = 1.0f;
+      bool rescale = false;
+      if (mx > -CUDART_INF_F) {
+        if (m_used == -CUDART_INF_F) {
+          m_used = mx;
+        } else if (mx > m_used + kRescaleLog2) {
+          alpha = exp2f(m_used - mx);
+          m_used = mx;
+          rescale = true;
+        }
+      }
+      float psum = 0.0f;
+      uint32_t ph[16], pl[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const float p0 = (s2[2 * k] == -CUDART_INF_F) ? 0.0f : exp2f(s2[2 * k] - m_used);
+        const float p1 = (s2[2 * k + 1] == -CUDART_INF_F) ? 0.0f : exp2f(s2[2 * k + 1] - m_used);
+        psum += p0 + p1;
+        __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+        const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+        __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - __uint_as_float(hw << 16),
+                                                  p1 - __uint_as_float(hw & 0xFFFF0000u));
+        ph[k] = hw;
+        pl[k] = *reinterpret_cast<uint32_t*>(&lb);
+      }
+      l_sum = l_sum * alpha + psum;
+
+      // P tile (this row) -> smem, once PV of chunk j-2 released the buffer
+      if (j >= 2 &&
+          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        ok = false;
+        break;
+      }
+      uint8_t* pt = smem + kOffP + sb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
+#pragma unroll
+      for (int kc = 0; kc < 4; ++kc) {
+        *reinterpret_cast<uint4*>(pt + kc * 128) = make_uint4(ph[4 * kc], ph[4 * kc + 1], ph[4 * kc + 2], ph[4 * kc + 3]);
+        *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
+            make_uint4(pl[4 * kc], pl[4 * kc + 1], pl[4 * kc + 2], pl[4 * kc + 3]);
+      }
+
+      // rescale this row's half of O in TMEM (warp-collective: lanes that do not
+      // need it multiply by 1); O must be quiescent: PV of chunk j-1 complete
+      if (__any_sync(0xffffffffu, rescale && o_live)) {
+        if (!__all_sync(kFull,
+                        ptx::mbar_wait(&bars.p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const float f = (rescale && o_live) ? alpha : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < kHalfC / 32; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+          ptx::tmem_st32(lane_base + kTmemO + c * 32, ov);
+        }
+        ptx::tmem_st_wait();
+      }
+      o_live = true;
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars.p_full[sb]);
+    }
+
+    // epilogue: O / l for this CTA's 256 channels
+    if (!ok) fail(a, abort_flag);
+    const bool o_ready = ptx::mbar_wait(bars.o_full, 0, abort_flag, kWaitLimitNs);
+    const int aborted = *abort_flag;
+    if (__all_sync(kFull, o_ready && ok && !aborted)) {  // warp-uniform: TMEM loads are collective
+      ptx::tc_fence_after();
+      const float inv = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
+      const float lse = l_sum > 0.0f ? (m_used + log2f(l_sum)) * kLn2 : -CUDART_INF_F;
+      const size_t part = (static_cast<size_t>(b) * a.n_split + split) * a.rows + row;
+#pragma unroll 1
+      for (int c = 0; c < kHalfC / 32; ++c) {
+        uint32_t ov[32];
+        ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+        ptx::tmem_ld_wait();
+        const int col = crank * kHalfC + c * 32;
+        if (!row_ok) continue;
+        if (a.n_split == 1 && !a.out_f32) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc + col);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(ov[8 * k + 2 * e]) * inv,
+                                                       __uint_as_float(ov[8 * k + 2 * e + 1]) * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float* base = (a.n_split == 1) ? static_cast<float*>(a.out) + qrow * kDc + col
+                                         : a.o_part + part * kDc + col;
+          float4* dst = reinterpret_cast<float4*>(base);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
+                                 __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
+        }
+      }
+      if (crank == 0 && row_ok) {
+        if (a.n_split == 1) {
+          if (a.lse) a.lse[qrow] = lse;
+        } else {
+          a.lse_part[part] = lse;
+        }
+      }
+    }
+  }
+
+  // ---- teardown ----
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+  ptx::cluster_sync();  // no remote store or arrive may target a CTA that has exited
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D byte tensor [pages][64 tokens][width bytes] at base (row stride = width,
+// page stride = page_bytes); box = box_w bytes x 32 tokens x 1 page.
+bool make_map(CUtensorMap* m, const void* base, int width, int box_w, int page_bytes, int num_pages,
+              CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(kPage),
+                              static_cast<cuuint64_t>(num_pages)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(page_bytes)};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_w), static_cast<cuuint32_t>(kChunk), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BC, int GC, int BR, int GR>
+cudaError_t launch_t(const DecodeLaunch& L) {
+  using G = QGeom<BC, GC, BR, GR>;
+  TmapSet tm;
+  const uint8_t* pool = static_cast<const uint8_t*>(L.pool);
+  const CUtensorMapSwizzle swz_c = (BC == 4) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map(&tm.cc, pool + G::kOffCC, G::kRowC, G::kRowC / 2, G::kPageBytes, L.num_pages, swz_c) ||
+      !make_map(&tm.rc, pool + G::kOffRC, G::kRowR, G::kRowR, G::kPageBytes, L.num_pages,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&tm.cm, pool + G::kOffCM, G::kGroupsC * 4, G::kGroupsC * 2, G::kPageBytes, L.num_pages,
+                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
+  const DecodeArgs a = make_decode_args(L);
+  const int row_tiles = (a.rows + kRows - 1) / kRows;
+  const long units = static_cast<long>(a.B) * a.n_split * row_tiles;
+  if (units * 2 > 0x7FFFFFFFL) return cudaErrorNotSupported;
+  auto kern = decode_tc_kernel<BC, GC, BR, GR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  if (e != cudaSuccess) return e;
+  const bool fast = (L.flags & MLA_DECODE_FAST_UNCOMPENSATED) != 0;
+  kern<<<static_cast<unsigned>(units * 2), kThreads, kSmemAlloc, L.stream>>>(a, tm, row_tiles, fast ? 1 : 2,
+                                                                             fast ? 1 : 3);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_decode_tc(const DecodeLaunch& L) {
+  if (!L.quantized || L.num_pages < 1) return cudaErrorNotSupported;
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
+      minor != 0)
+    return cudaErrorNotSupported;
+#define MLA_TC_CASE(BC, GC, BR, GR)                                              \
+  if (L.bits_c == BC && L.group_c == GC && L.bits_r == BR && L.group_r == GR)  \
+    return tc::launch_t<BC, GC, BR, GR>(L);
+#define MLA_TC_R(BC, GC) \
+  MLA_TC_CASE(BC, GC, 4, 64) MLA_TC_CASE(BC, GC, 4, 32) MLA_TC_CASE(BC, GC, 2, 64) MLA_TC_CASE(BC, GC, 2, 32)
+  MLA_TC_R(4, 64)
+  MLA_TC_R(4, 32)
+  MLA_TC_R(2, 64)
+  MLA_TC_R(2, 32)
+#undef MLA_TC_R
+#undef MLA_TC_CASE
+  return cudaErrorNotSupported;
+}
 
 }  // namespace mla

@@ -46,12 +46,11 @@ def test_append_extreme_values_bit_exact():
     toks[3, :] = -0.0
     toks[3, 7] = 0.25
     toks[4] = rng.standard_normal(576) * np.exp(rng.normal(0, 3, 576))
-    toks[5, :64] = 65504.0
-    toks[5, 64:] = -65504.0
+    toks[5, :64] = 65280.0   # the largest bf16 value within fp16's range
+    toks[5, 64:] = -65280.0
     toks[6] = np.where(rng.random(576) < 0.5, -1e-7, 3e-8)
     toks[7] = rng.standard_normal(576)
-    toks = np.clip(toks, -65504, 65504)
-    bits = synth.f32_to_bf16_bits(toks)
+    bits = synth.f32_to_bf16_bits(np.clip(toks, -65280, 65280))
     x = synth.bf16_bits_to_f32(bits)
     for bc, gc, br, gr in BIT_COMBOS:
         desc = api.make_desc(bc, gc, br, gr, num_pages=1)
