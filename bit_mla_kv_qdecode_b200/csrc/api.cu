@@ -57,9 +57,11 @@ struct SplitPlan {
 };
 
 // Split each request's pages into n page-aligned chunks. An explicit request
-// is honoured (capped at the page count). The automatic choice aims at about
-// two waves of 128-row work units over the SMs, and never cuts a request into
-// chunks shorter than 4 pages.
+// is honoured (capped at the page count). The automatic choice models the
+// decode time of the longest request as waves(n) * (pages / n), where a wave
+// is one work unit (128 query rows of one request and one split) on each
+// 2-CTA cluster slot, and picks the smallest n within 3% of the best, with
+// chunks of at least 4 pages.
 SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
   const int pages = std::max(1, (max_seq_len + mla::kPage - 1) / mla::kPage);
   int n;
@@ -67,10 +69,18 @@ SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
     n = std::min(requested, pages);
   } else {
     const long units = static_cast<long>(std::max(B, 1)) * ((static_cast<long>(s_q) * H + 127) / 128);
-    const long slots = device_sm_count() / 2;  // one 2-CTA cluster per unit
-    long want = (2 * slots + units - 1) / units;
-    want = std::min<long>(want, (pages + 3) / 4);
-    n = static_cast<int>(std::max<long>(1, want));
+    const long slots = std::max(1, device_sm_count() / 2);
+    const int n_max = std::max(1, std::min(pages / 4, 64));
+    double best = 1e30;
+    n = 1;
+    for (int c = 1; c <= n_max; ++c) {
+      const long waves = (units * c + slots - 1) / slots;
+      const double cost = static_cast<double>(waves) * ((pages + c - 1) / c) + 2.0 * waves;  // + per-unit overhead
+      if (cost < best * 0.97) {
+        best = cost;
+        n = c;
+      }
+    }
   }
   const int chunk = (pages + n - 1) / n;
   return SplitPlan{(pages + chunk - 1) / chunk, chunk};

@@ -26,7 +26,9 @@
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: packed codes + metadata of 32-token chunks
-//   warp 1      TMEM owner and the single MMA-issuing thread
+//   warp 1      TMEM owner; issues the QK MMAs of even chunks
+//   warp 6      issues the PV MMAs
+//   warp 7      issues the QK MMAs of odd chunks
 //   warps 2-5   unpack + dequantize into bf16 hi/lo operand tiles
 //   warps 8-11  one thread per row: score exchange, online softmax, P tiles,
 //               output rescaling in TMEM, epilogue
@@ -58,13 +60,17 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // TMEM columns
 constexpr uint32_t kTmemO = 0;        // 256 fp32 columns: this CTA's half of O
-constexpr uint32_t kTmemS = 256;      // two 32-column score buffers
-constexpr uint32_t kTmemQ = 320;      // 144 columns: Q (288 bf16 per row)
+constexpr uint32_t kTmemS = 256;      // two 64-column score buffers: [S_hi | S_lo] of 32 tokens
+constexpr uint32_t kTmemQ = 384;      // 128 columns: content part of Q (256 bf16 per row)
 constexpr uint32_t kTmemCols = 512;
 
 // Shared memory layout (bytes)
-constexpr int kCTile = kKChunks * 4 * 128;         // one bf16 operand tile: 36 chunks x 4 token groups x 128 B
-constexpr int kCStage = 2 * kCTile;                // hi + lo
+// Operand stage: per 8-channel chunk c, the hi and lo core matrices of the 32
+// tokens sit side by side ([c][hi/lo][token group][8 rows x 16 B]), so one
+// K-major QK operand of N = 64 rows covers C_hi and C_lo of the same tokens.
+constexpr int kCChunkStride = 1024;
+constexpr int kCLoOff = 512;
+constexpr int kCStage = kKChunks * kCChunkStride;
 constexpr int kPTile = (kRows / 8) * 4 * 128;      // 8 KB: 16 row groups x 4 token groups x 128 B
 constexpr int kXRow = 36;                          // floats per row in the score-exchange buffer
 constexpr int kXBuf = kRows * kXRow * 4;
@@ -76,9 +82,11 @@ constexpr int kOffC = 0;
 constexpr int kOffP = kOffC + kNC * kCStage;
 constexpr int kOffX = kOffP + 2 * 2 * kPTile;
 constexpr int kOffCode = kOffX + 2 * kXBuf;
-constexpr int kOffBar = kOffCode + kNS * kCodeStage;
-constexpr int kNumBars = 2 * kNS + 2 * kNC + 2 + 2 + 2 + 2 + 2 + 2 + 2;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kOffBar = kOffCode + kNS * kCodeStage + kRows * kHalfR * 2;
+constexpr int kOffQR = kOffCode + kNS * kCodeStage;  // rope part of Q: 128 rows x 32 bf16, core matrices
+constexpr int kQRBytes = kRows * kHalfR * 2;
+constexpr int kNumBars = 2 * kNS + 2 * kNC + 16;
+constexpr int kOffMisc = kOffQR + kQRBytes + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;      // slack to align the base to 1024
 static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0, "TMA swizzle needs 1024-byte aligned stages");
@@ -101,9 +109,10 @@ struct Bars {
   uint64_t* p_full;      // [2] softmax P tile + O rescale -> MMA
   uint64_t* p_empty;     // [2] MMA (PV) -> softmax
   uint64_t* x_full;      // [2] peer wrote its partial scores into my exchange buffer
-  uint64_t* x_empty;     // [2] peer consumed what I wrote into its exchange buffer
   uint64_t* q_full;      // [1] Q in TMEM
-  uint64_t* o_full;      // [1] all MMAs of the unit done
+  uint64_t* o_full;      // [1] all PV MMAs of the unit done
+  uint64_t* qk_drain;    // [1] all QK MMAs of the even-chunk issuer done
+  uint64_t* qk_drain2;   // [1] ... of the odd-chunk issuer
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
@@ -119,9 +128,10 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.p_full = p + 4;
   r.p_empty = p + 6;
   r.x_full = p + 8;
-  r.x_empty = p + 10;
   r.q_full = p + 12;
   r.o_full = p + 13;
+  r.qk_drain = p + 14;
+  r.qk_drain2 = p + 15;
   return r;
 }
 
@@ -152,6 +162,54 @@ __device__ __forceinline__ void dequant8(uint32_t w, float s, float z, float (&x
   for (int k = 0; k < 8; ++k) x[k] = fmaf(u2f((w >> (k * BITS)) & mask), s, z);
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {  // 2^x; -inf -> +0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 8 codes of one word -> bf16 hi/lo of u*s+z, with packed fp32x2 arithmetic.
+// Code k sits at bits [k*BITS, (k+1)*BITS). Each code is placed in the low
+// byte of the float 2^23 (exact integer embedding), the 2^23 is subtracted,
+// and u*s+z is one fused multiply-add per pair.
+template <int BITS>
+__device__ __forceinline__ void dequant_split8(uint32_t w, float2 s2, float2 z2, uint4& hi, uint4& lo) {
+  uint32_t b[8];
+  if constexpr (BITS == 4) {
+    const uint32_t ev = w & 0x0F0F0F0Fu, od = (w >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 / 1,3,5,7 in bytes
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      b[2 * k] = __byte_perm(ev, 0x4B000000u, 0x7650 | k);
+      b[2 * k + 1] = __byte_perm(od, 0x4B000000u, 0x7650 | k);
+    }
+  } else {
+    const uint32_t q0 = w & 0x03030303u, q1 = (w >> 2) & 0x03030303u;  // codes 0,4 / 1,5 in bytes 0,1 ...
+    const uint32_t q2 = (w >> 4) & 0x03030303u, q3 = (w >> 6) & 0x03030303u;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      b[4 * k] = __byte_perm(q0, 0x4B000000u, 0x7650 | k);
+      b[4 * k + 1] = __byte_perm(q1, 0x4B000000u, 0x7650 | k);
+      b[4 * k + 2] = __byte_perm(q2, 0x4B000000u, 0x7650 | k);
+      b[4 * k + 3] = __byte_perm(q3, 0x4B000000u, 0x7650 | k);
+    }
+  }
+  const float2 magic = make_float2(-8388608.0f, -8388608.0f);
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float2 u = __fadd2_rn(make_float2(__uint_as_float(b[2 * k]), __uint_as_float(b[2 * k + 1])), magic);
+    const float2 x = __ffma2_rn(u, s2, z2);
+    __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
+    const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
+    __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
+    h[k] = hw;
+    l[k] = *reinterpret_cast<uint32_t*>(&lb);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
 __device__ __forceinline__ void fail(const DecodeArgs& a, volatile int* abort_flag) {
   record_error(a.status, MLA_ERR_TIMEOUT);
   *abort_flag = 1;
@@ -167,6 +225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const Bars bars = carve_bars(smem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
+  volatile int* stage_page = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);  // [kNS]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t crank = ptx::cluster_ctarank();
@@ -224,11 +283,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars.s_empty[i], 128);
       ptx::mbar_init(&bars.p_full[i], 128);
       ptx::mbar_init(&bars.p_empty[i], 1);
-      ptx::mbar_init(&bars.x_full[i], 128);
-      ptx::mbar_init(&bars.x_empty[i], 128);
+      ptx::mbar_init(&bars.x_full[i], 1);     // armed locally with expect_tx; bytes come from the peer
     }
     ptx::mbar_init(bars.q_full, 128);
     ptx::mbar_init(bars.o_full, 1);
+    ptx::mbar_init(bars.qk_drain, 1);
+    ptx::mbar_init(bars.qk_drain2, 1);
     *abort_flag = 0;
     ptx::fence_mbar_init_cluster();
   }
@@ -263,6 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int t0 = t_begin + j * kChunk;
         const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
         uint8_t* st = smem + kOffCode + s * kCodeStage;
+        stage_page[s] = page;  // published to the dequant warps by the release-arrive below
         if (page >= 0) {
           ptx::mbar_arrive_expect_tx(&bars.code_full[s], bytes);
           const int slot0 = t0 % kPage;
@@ -283,61 +344,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kNS; ++s)
         if (issued[s] > 0) ptx::mbar_wait(&bars.code_full[s], ((issued[s] - 1) / kNS) & 1, nullptr, kWaitLimitNs);
     }
-  } else if (warp == 1) {
-    // =========================== MMA issuer ===========================
+  } else if (warp == 1 || warp == 7) {
+    // =========================== QK issuers ===========================
+    // S_j[128 rows x 64] = Q . [C_hi ; C_lo]^T over this CTA's 288 channels:
+    // 16 K-steps with the content part of Q in TMEM, 2 with its RoPE part in
+    // shared memory. Descriptors are built once; K-steps only move the start
+    // address field.
+    // Two issuing threads (even / odd chunks) hide the per-instruction issue
+    // latency of tcgen05.mma; each owns one of the two score buffers.
     if (lane == 0) {
-      const uint32_t idesc_qk = ptx::idesc_bf16_f32(kRows, kChunk, 0, 0);
-      const uint32_t idesc_pv = ptx::idesc_bf16_f32(kRows, kHalfC, 0, 1);
-      const uint32_t c_base = ptx::smem_u32(smem + kOffC);
-      const uint32_t p_base = ptx::smem_u32(smem + kOffP);
+      const int par = (warp == 1) ? 0 : 1;
+      uint64_t* drain = (warp == 1) ? bars.qk_drain : bars.qk_drain2;
+      const uint32_t idesc = ptx::idesc_bf16_f32(kRows, n_terms_qk == 2 ? 2 * kChunk : kChunk, 0, 0);
+      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), kCChunkStride, 128);
+      const uint64_t a_rope = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffQR), 128, 512);
       bool ok = ptx::mbar_wait(bars.q_full, 0, abort_flag, kWaitLimitNs);
-      ptx::tc_fence_after();
-      auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1, cs = j % kNC;
-        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) return false;
-        ptx::tc_fence_after();
-        const uint32_t pt = p_base + pb * 2 * kPTile;
-        const uint32_t ct = c_base + cs * kCStage;
-        for (int term = 0; term < n_terms_pv; ++term) {
-          const uint32_t pa = pt + (term == 1 ? kPTile : 0);     // P_lo for term 1
-          const uint32_t cb = ct + (term == 2 ? kCTile : 0);     // C_lo for term 2
-#pragma unroll
-          for (int k = 0; k < kChunk / 16; ++k) {
-            const uint64_t ad = ptx::smem_desc_noswizzle(pa + k * 256, 128, 512);
-            const uint64_t bd = ptx::smem_desc_noswizzle(cb + k * 256, 128, 512);
-            ptx::mma_ss(tmem + kTmemO, ad, bd, idesc_pv, (j > 0 || term > 0 || k > 0) ? 1u : 0u);
-          }
-        }
-        ptx::mma_commit(&bars.p_empty[pb]);
-        ptx::mma_commit(&bars.c_empty[cs]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_chunks; ++j) {
+      for (int j = par; ok && j < n_chunks; j += 2) {
         const int cs = j % kNC, sb = j & 1;
-        if (!ptx::mbar_wait(&bars.c_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        if (j >= 2 && !ptx::mbar_wait(&bars.s_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait(&bars.c_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs) ||
+            (j >= 2 && !ptx::mbar_wait(&bars.s_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t ct = c_base + cs * kCStage;
-        for (int term = 0; term < n_terms_qk; ++term) {
-          const uint32_t cb = ct + term * kCTile;
-#pragma unroll 6
-          for (int k = 0; k < kKChunks / 2; ++k) {
-            const uint64_t bd = ptx::smem_desc_noswizzle(cb + k * 2 * 512, 512, 128);
-            ptx::mma_ts(tmem + kTmemS + sb * kChunk, tmem + kTmemQ + k * 8, bd, idesc_qk,
-                        (term > 0 || k > 0) ? 1u : 0u);
-          }
-        }
+        const uint64_t bs = b0 + static_cast<uint64_t>((cs * kCStage) >> 4);
+        const uint32_t d = tmem + kTmemS + sb * 2 * kChunk;
+#pragma unroll
+        for (int k = 0; k < kHalfC / 16; ++k)
+          ptx::mma_ts(d, tmem + kTmemQ + k * 8, bs + static_cast<uint64_t>((k * 2 * kCChunkStride) >> 4), idesc,
+                      k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < kHalfR / 16; ++k)
+          ptx::mma_ss(d, a_rope + static_cast<uint64_t>((k * 256) >> 4),
+                      bs + static_cast<uint64_t>(((kHalfC / 8 + 2 * k) * kCChunkStride) >> 4), idesc, 1u);
         ptx::mma_commit(&bars.s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
-      if (ok) ok = issue_pv(n_chunks - 1);
+      if (!ok) fail(a, abort_flag);
+      ptx::mma_commit(drain);
+      ptx::mbar_wait(drain, 0, nullptr, kWaitLimitNs);  // MMAs finish before TMEM is released
+    }
+  } else if (warp == 6) {
+    // =========================== PV issuer ===========================
+    // O_half[128 x 256] += P_hi.C_hi + P_lo.C_hi + P_hi.C_lo over the chunk's 32 tokens.
+    if (lane == 0) {
+      const uint32_t idesc = ptx::idesc_bf16_f32(kRows, kHalfC, 0, 1);
+      const uint64_t a0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffP), 128, 512);
+      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), 128, kCChunkStride);
+      bool ok = true;
+      for (int j = 0; j < n_chunks; ++j) {
+        const int pb = j & 1, cs = j % kNC;
+        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint64_t ap = a0 + static_cast<uint64_t>((pb * 2 * kPTile) >> 4);
+        const uint64_t bc = b0 + static_cast<uint64_t>((cs * kCStage) >> 4);
+        for (int term = 0; term < n_terms_pv; ++term) {
+          const uint64_t at = ap + (term == 1 ? static_cast<uint64_t>(kPTile >> 4) : 0);   // P_lo for term 1
+          const uint64_t bt = bc + (term == 2 ? static_cast<uint64_t>(kCLoOff >> 4) : 0);  // C_lo for term 2
+#pragma unroll
+          for (int k = 0; k < kChunk / 16; ++k)
+            ptx::mma_ss(tmem + kTmemO, at + static_cast<uint64_t>((k * 256) >> 4),
+                        bt + static_cast<uint64_t>((k * 256) >> 4), idesc, (j > 0 || term > 0 || k > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(&bars.p_empty[pb]);
+        ptx::mma_commit(&bars.c_empty[cs]);
+      }
       if (!ok) fail(a, abort_flag);
       ptx::mma_commit(bars.o_full);
-      // every issued MMA must finish before TMEM is released, abort or not
-      ptx::mbar_wait(bars.o_full, 0, nullptr, kWaitLimitNs);
+      ptx::mbar_wait(bars.o_full, 0, nullptr, kWaitLimitNs);  // MMAs finish before TMEM is released
     }
   } else if (warp >= 2 && warp < 6) {
     // =========================== dequant ===========================
@@ -352,10 +428,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       const int t0 = t_begin + j * kChunk;
-      const bool valid = (t0 + tq < t_end) && lookup_page(a.table, a.max_pages, a.num_pages, b, t0) >= 0;
+      const bool valid = (t0 + tq < t_end) && stage_page[s] >= 0;
       const uint8_t* st = smem + kOffCode + s * kCodeStage;
       uint8_t* chi = smem + kOffC + cs * kCStage;
-      uint8_t* clo = chi + kCTile;
+      uint8_t* clo = chi + kCLoOff;
       // content: quads qsel and qsel+4 (32 channels each)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -375,12 +451,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
-          if (valid) {
-            float x[8];
-            dequant8<BITS_C>(w[i], sc, zc, x);
-            split8(x, hi, lo);
-          }
-          const int off = (4 * q + i) * 512 + tq * 16;
+          if (valid) dequant_split8<BITS_C>(w[i], make_float2(sc, sc), make_float2(zc, zc), hi, lo);
+          const int off = (4 * q + i) * kCChunkStride + tq * 16;
           *reinterpret_cast<uint4*>(chi + off) = hi;
           *reinterpret_cast<uint4*>(clo + off) = lo;
         }
@@ -393,12 +465,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t w = (BITS_R == 4) ? *reinterpret_cast<const uint32_t*>(row + qsel * 4)
                                          : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + qsel * 2));
         uint4 hi = make_uint4(0, 0, 0, 0), lo = hi;
-        if (valid) {
-          float x[8];
-          dequant8<BITS_R>(w, sr, zr, x);
-          split8(x, hi, lo);
-        }
-        const int off = (32 + qsel) * 512 + tq * 16;
+        if (valid) dequant_split8<BITS_R>(w, make_float2(sr, sr), make_float2(zr, zr), hi, lo);
+        const int off = (32 + qsel) * kCChunkStride + tq * 16;
         *reinterpret_cast<uint4*>(chi + off) = hi;
         *reinterpret_cast<uint4*>(clo + off) = lo;
       }
@@ -415,154 +483,193 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const size_t qrow = static_cast<size_t>(b) * a.rows + (row_ok ? row : 0);
 
-    // Q half -> TMEM columns [320, 464) (zeros for padding rows)
+    // Q: content half -> TMEM columns [384, 512); RoPE half -> shared memory
+    // (K-major core matrices, the A operand of the two RoPE K-steps).
+    // Padding rows get zeros.
     {
       const uint4* qc = reinterpret_cast<const uint4*>(a.q_c + qrow * kDc + crank * kHalfC);
       const uint4* qr = reinterpret_cast<const uint4*>(a.q_r + qrow * kDr + crank * kHalfR);
 #pragma unroll
-      for (int blk = 0; blk < 5; ++blk) {
+      for (int blk = 0; blk < 4; ++blk) {
         uint32_t v[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int c16 = blk * 8 + k;  // 16-byte piece (8 bf16) index, 36 pieces
-          uint4 x = make_uint4(0, 0, 0, 0);
-          if (row_ok && c16 < 32) x = __ldg(qc + c16);
-          else if (row_ok && c16 < 36) x = __ldg(qr + (c16 - 32));
+          const uint4 x = row_ok ? __ldg(qc + blk * 8 + k) : make_uint4(0, 0, 0, 0);
           v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
         }
         ptx::tmem_st32(lane_base + kTmemQ + blk * 32, v);
       }
+      uint8_t* qrs = smem + kOffQR + (i >> 3) * 512 + (i & 7) * 16;
+#pragma unroll
+      for (int kc = 0; kc < 4; ++kc)
+        *reinterpret_cast<uint4*>(qrs + kc * 128) = row_ok ? __ldg(qr + kc) : make_uint4(0, 0, 0, 0);
+      ptx::fence_proxy_async_smem();
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bars.q_full);
     }
 
-    const uint32_t xbuf_local = ptx::smem_u32(smem + kOffX);
-    const uint32_t xbuf_peer = ptx::mapa(xbuf_local, peer);
+    // Score exchange. Step j first finishes chunk j-1 (its peer half arrived
+    // during the previous step), then reads this CTA's partial S_j from TMEM
+    // and stores it into the peer's exchange buffer with st.async, which
+    // completes bytes on the peer's x_full. Two buffers suffice without any
+    // release handshake: the peer sends chunk j-1 only after it has read
+    // chunk j-2, and this thread sees chunk j-1 arrive before it sends chunk j
+    // into the buffer chunk j-2 used.
+    const uint32_t xbuf_peer = ptx::mapa(ptx::smem_u32(smem + kOffX), peer);
     const uint32_t xfull_peer = ptx::mapa(ptx::smem_u32(bars.x_full), peer);
-    const uint32_t xempty_peer = ptx::mapa(ptx::smem_u32(bars.x_empty), peer);
     float m_used = -CUDART_INF_F, l_sum = 0.0f;
     bool o_live = false;  // O has been written by a PV MMA
     bool ok = true;
+    uint32_t prev[32];
+    bool prev_page_ok = false;
 
-    for (int j = 0; j < n_chunks && ok; ++j) {
-      const int sb = j & 1;
-      const int t0 = t_begin + j * kChunk;
-      // wait results are made warp-uniform: the TMEM loads below are warp-collective
-      if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      uint32_t sv[32];
-      ptx::tmem_ld32(lane_base + kTmemS + sb * kChunk, sv);
-      ptx::tmem_ld_wait();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars.s_empty[sb]);
-
-      // exchange partial scores with the peer CTA
-      if (j >= 2 &&
-          !__all_sync(kFull, ptx::mbar_wait<true>(&bars.x_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      const uint32_t my_row_peer = xbuf_peer + sb * kXBuf + i * (kXRow * 4);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        ptx::st_cluster_v4(my_row_peer + k * 16, __uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1]),
-                           __uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3]));
-      ptx::mbar_arrive_remote(xfull_peer + sb * 8);
-      if (!__all_sync(kFull, ptx::mbar_wait<true>(&bars.x_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + sb * kXBuf + i * (kXRow * 4));
-      float s2[32];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float4 pv = xr[k];
-        s2[4 * k] = __uint_as_float(sv[4 * k]) + pv.x;
-        s2[4 * k + 1] = __uint_as_float(sv[4 * k + 1]) + pv.y;
-        s2[4 * k + 2] = __uint_as_float(sv[4 * k + 2]) + pv.z;
-        s2[4 * k + 3] = __uint_as_float(sv[4 * k + 3]) + pv.w;
-      }
-      ptx::mbar_arrive_remote(xempty_peer + sb * 8);
-
-      // mask + scale (log2 domain)
-      const bool page_ok = lookup_page(a.table, a.max_pages, a.num_pages, b, t0) >= 0;
-      const int lim = page_ok ? min(L, t_end) - t0 : 0;
-      float mx = -CUDART_INF_F;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        s2[k] = (k < lim) ? s2[k] * a.scale_log2 : -CUDART_INF_F;
-        mx = fmaxf(mx, s2[k]);
-      }
-      float alpha = 1.0f;
-      bool rescale = false;
-      if (mx > -CUDART_INF_F) {
-        if (m_used == -CUDART_INF_F) {
-          m_used = mx;
-        } else if (mx > m_used + kRescaleLog2) {
-          alpha = exp2f(m_used - mx);
-          m_used = mx;
-          rescale = true;
+    for (int j = 0; j <= n_chunks && ok; ++j) {
+      if (j >= 1) {
+        const int jj = j - 1, pb = jj & 1;
+        const int t0 = t_begin + jj * kChunk;
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.x_full[pb], (jj >> 1) & 1, abort_flag, kWaitLimitNs))) {
+          ok = false;
+          break;
         }
-      }
-      float psum = 0.0f;
-      uint32_t ph[16], pl[16];
+        const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + pb * kXBuf + i * (kXRow * 4));
+        // full score = my partial + peer partial, then * scale * log2(e)
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+        float2 sp[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float p0 = (s2[2 * k] == -CUDART_INF_F) ? 0.0f : exp2f(s2[2 * k] - m_used);
-        const float p1 = (s2[2 * k + 1] == -CUDART_INF_F) ? 0.0f : exp2f(s2[2 * k + 1] - m_used);
-        psum += p0 + p1;
-        __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-        const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
-        __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - __uint_as_float(hw << 16),
-                                                  p1 - __uint_as_float(hw & 0xFFFF0000u));
-        ph[k] = hw;
-        pl[k] = *reinterpret_cast<uint32_t*>(&lb);
-      }
-      l_sum = l_sum * alpha + psum;
-
-      // P tile (this row) -> smem, once PV of chunk j-2 released the buffer
-      if (j >= 2 &&
-          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
-        ok = false;
-        break;
-      }
-      uint8_t* pt = smem + kOffP + sb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
+        for (int k = 0; k < 8; ++k) {
+          const float4 pv = xr[k];
+          sp[2 * k] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k]), __uint_as_float(prev[4 * k + 1])),
+                                            make_float2(pv.x, pv.y)), sc2);
+          sp[2 * k + 1] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k + 2]),
+                                                            __uint_as_float(prev[4 * k + 3])),
+                                                make_float2(pv.z, pv.w)), sc2);
+        }
+        const int lim = prev_page_ok ? min(L, t_end) - t0 : 0;
+        if (lim < kChunk) {  // partially visible chunk (ragged tail, causal row, bad page)
 #pragma unroll
-      for (int kc = 0; kc < 4; ++kc) {
-        *reinterpret_cast<uint4*>(pt + kc * 128) = make_uint4(ph[4 * kc], ph[4 * kc + 1], ph[4 * kc + 2], ph[4 * kc + 3]);
-        *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
-            make_uint4(pl[4 * kc], pl[4 * kc + 1], pl[4 * kc + 2], pl[4 * kc + 3]);
-      }
+          for (int k = 0; k < 16; ++k) {
+            if (2 * k >= lim) sp[k].x = -CUDART_INF_F;
+            if (2 * k + 1 >= lim) sp[k].y = -CUDART_INF_F;
+          }
+        }
+        float mt[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) mt[k] = fmaxf(sp[k].x, sp[k].y);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) mt[k] = fmaxf(mt[k], mt[k + w]);
+        const float mx = mt[0];
+        float alpha = 1.0f;
+        bool rescale = false;
+        if (mx > -CUDART_INF_F) {
+          if (m_used == -CUDART_INF_F) {
+            m_used = mx;
+          } else if (mx > m_used + kRescaleLog2) {
+            alpha = ex2_approx(m_used - mx);
+            m_used = mx;
+            rescale = true;
+          }
+        }
+        // p = 2^(s - m); rows that have seen no key use m = 0, so every p is 0
+        const float m_eff = (m_used == -CUDART_INF_F) ? 0.0f : m_used;
+        const float2 negm = make_float2(-m_eff, -m_eff);
+        uint32_t ph[16], pl[16];
+        float2 ps[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 d = __fadd2_rn(sp[k], negm);
+          const float2 pk = make_float2(ex2_approx(d.x), ex2_approx(d.y));
+          ps[k] = pk;
+          __nv_bfloat162 hb = __floats2bfloat162_rn(pk.x, pk.y);
+          const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+          const float2 r = __fadd2_rn(pk, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
+          __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
+          ph[k] = hw;
+          pl[k] = *reinterpret_cast<uint32_t*>(&lb);
+        }
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) ps[k] = __fadd2_rn(ps[k], ps[k + w]);
+        const float psum = ps[0].x + ps[0].y;
+        l_sum = l_sum * alpha + psum;
 
-      // rescale this row's half of O in TMEM (warp-collective: lanes that do not
-      // need it multiply by 1); O must be quiescent: PV of chunk j-1 complete
-      if (__any_sync(0xffffffffu, rescale && o_live)) {
-        if (!__all_sync(kFull,
-                        ptx::mbar_wait(&bars.p_empty[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        // P tile (this row) -> smem, once PV of chunk jj-2 released the buffer
+        if (jj >= 2 &&
+            !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
+#pragma unroll
+        for (int kc = 0; kc < 4; ++kc) {
+          *reinterpret_cast<uint4*>(pt + kc * 128) =
+              make_uint4(ph[4 * kc], ph[4 * kc + 1], ph[4 * kc + 2], ph[4 * kc + 3]);
+          *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
+              make_uint4(pl[4 * kc], pl[4 * kc + 1], pl[4 * kc + 2], pl[4 * kc + 3]);
+        }
+
+        // rescale this row's half of O in TMEM (warp-collective: lanes that do
+        // not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
+        if (__any_sync(kFull, rescale && o_live)) {
+          if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
+                                                kWaitLimitNs))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const float f = (rescale && o_live) ? alpha : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < kHalfC / 32; ++c) {
+            uint32_t ov[32];
+            ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+            ptx::tmem_st32(lane_base + kTmemO + c * 32, ov);
+          }
+          ptx::tmem_st_wait();
+        }
+        o_live = true;
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars.p_full[pb]);
+      }
+      uint32_t cur[32];
+      bool cur_page_ok = false;
+      if (j < n_chunks) {
+        const int sb = j & 1;
+        // wait results are made warp-uniform: the TMEM loads below are warp-collective
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        const float f = (rescale && o_live) ? alpha : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < kHalfC / 32; ++c) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+        ptx::tmem_ld32(lane_base + kTmemS + sb * 2 * kChunk, cur);
+        if (n_terms_qk == 2) {  // add the C_lo half of the score tile
+          uint32_t lo[32];
+          ptx::tmem_ld32(lane_base + kTmemS + sb * 2 * kChunk + kChunk, lo);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-          ptx::tmem_st32(lane_base + kTmemO + c * 32, ov);
+          for (int k = 0; k < 32; ++k) cur[k] = __float_as_uint(__uint_as_float(cur[k]) + __uint_as_float(lo[k]));
         }
-        ptx::tmem_st_wait();
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars.s_empty[sb]);
+        // page validity of chunk j, consumed one step later (hides the load)
+        cur_page_ok = lookup_page(a.table, a.max_pages, a.num_pages, b, t_begin + j * kChunk) >= 0;
+        if (i == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kRows * kChunk * 4);
+        const uint32_t dst = xbuf_peer + sb * kXBuf + i * (kXRow * 4);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ptx::st_async_v4(dst + k * 16, cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3],
+                           xfull_peer + sb * 8);
       }
-      o_live = true;
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars.p_full[sb]);
+#pragma unroll
+      for (int k = 0; k < 32; ++k) prev[k] = cur[k];
+      prev_page_ok = cur_page_ok;
     }
 
     // epilogue: O / l for this CTA's 256 channels
