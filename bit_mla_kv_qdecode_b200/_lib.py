@@ -26,6 +26,8 @@ MLA_DECODE_DEFAULT = 0
 MLA_DECODE_FORCE_SIMT = 1
 MLA_DECODE_FAST_UNCOMPENSATED = 2
 
+MLA_QDECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
+
 
 class mla_qcache_desc(ctypes.Structure):
     _fields_ = [(n, _c_int) for n in ("d_c", "d_r", "bits_c", "group_c", "bits_r", "group_r",
@@ -53,6 +55,8 @@ SIGNATURES = {
     "mla_decode_bf16": (_c_int, [_c_void, _c_int, _c_int, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void,
                                  _c_int, _c_int, _c_int, _c_float, _c_int, _c_void, _c_size, _c_void, _c_int,
                                  _c_void, _c_uint, _c_void]),
+    "mla_qdecode_noalloc": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void, _c_int,
+                                     _c_int, _c_int, _c_float, _c_int, _c_void, _c_int, _c_void, _c_uint, _c_void]),
     "mla_get_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_void]),
 }
 

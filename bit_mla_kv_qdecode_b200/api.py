@@ -119,6 +119,22 @@ def mla_qdecode(desc, pool, block_table, seq_lens, max_seq_len, q_c, q_r, scale,
     return out, lse
 
 
+def mla_qdecode_noalloc(desc, pool, block_table, seq_lens, max_seq_len, q_c, q_r, scale, out, lse=None, *,
+                        num_splits=0, flags=0, stream=None):
+    """mla_qdecode without a workspace argument, for callers that cannot
+    allocate: the split-KV scratch is a fixed array inside the library (see
+    include/mla_qcache.h). `out` must be given; nothing is allocated here."""
+    B, s_q, H = q_c.shape[:3]
+    f32 = {torch.float32: 1, torch.bfloat16: 0}[out.dtype]
+    check("mla_qdecode_noalloc", _lib.load().mla_qdecode_noalloc(
+        ctypes.byref(desc), _need(pool, "pool", torch.uint8), _need(block_table, "block_table", torch.int32),
+        block_table.shape[1], _need(seq_lens, "seq_lens", torch.int32, (B,)), int(max_seq_len),
+        _need(q_c, "q_c", torch.bfloat16, (B, s_q, H, D_C)), _need(q_r, "q_r", torch.bfloat16, (B, s_q, H, D_R)),
+        B, s_q, H, float(scale), int(num_splits), _need(out, "out", out.dtype, (B, s_q, H, D_C)), f32,
+        None if lse is None else _need(lse, "lse", torch.float32, (B, s_q, H)), int(flags), _stream(stream)))
+    return out, lse
+
+
 def mla_decode_bf16(pool, block_table, seq_lens, max_seq_len, q_c, q_r, scale, *, out=None,
                     out_dtype=torch.bfloat16, lse=None, num_splits=0, workspace=None, flags=0, stream=None):
     (B, s_q, H), qc, qr, out, po, pl, pw, nw, f32, _ = _decode_io(

@@ -31,7 +31,8 @@
  * -----------
  *  * The caller owns every buffer (pool, block table, queries, outputs,
  *    workspace). The library allocates no device memory; its only state is
- *    one device status word per GPU (see mla_get_device_status).
+ *    one device status word per GPU (see mla_get_device_status) and the
+ *    fixed scratch array of mla_qdecode_noalloc.
  *  * All pointers named "device" must be device memory (or memory the device
  *    can address) of the current CUDA device. "host" pointers are CPU memory.
  *  * Every call that takes a stream is asynchronous on that stream. Argument
@@ -211,6 +212,35 @@ mla_status mla_decode_bf16(const void* pool, int num_pages, int page_size,
                            void* workspace, size_t workspace_bytes,
                            void* out, int out_dtype, float* lse,
                            unsigned flags, mla_stream_t stream);
+
+/* Scratch held by every GPU that loads this library for mla_qdecode_noalloc. */
+#define MLA_QDECODE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* mla_qdecode for callers that cannot allocate device memory when they
+ * decode (a serving loop with a fixed memory budget that forbids allocation
+ * after start-up, a plug-in whose host framework owns all device memory,
+ * latency-critical code where an allocation could synchronise the device).
+ * The paper has no counterpart; it is a packaging choice of this library.
+ *   Arguments are those of mla_qdecode without the workspace: the split-KV
+ *   scratch comes from a fixed array of MLA_QDECODE_NOALLOC_SCRATCH_BYTES
+ *   compiled into the library (one per GPU, held until the process exits).
+ *   The caller still provides every input and output buffer.
+ *   Returns MLA_ERR_WORKSPACE, before launching anything, when the shape
+ *   needs more scratch than that (mla_decode_workspace_bytes tells how much);
+ *   otherwise the results and errors of mla_qdecode. It calls no allocator.
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Every call on a device shares the one array (it keeps the last call's
+ *   contents, and nothing in it needs clearing): calls whose executions
+ *   overlap on the GPU -- on different streams, or from different host
+ *   threads -- race on it and must be serialised by the caller. */
+mla_status mla_qdecode_noalloc(const mla_qcache_desc* desc, const void* pool,
+                               const int32_t* block_table, int max_pages_per_seq,
+                               const int32_t* seq_lens, int max_seq_len,
+                               const void* q_c, const void* q_r,
+                               int B, int s_q, int H, float scale, int num_splits,
+                               void* out, int out_dtype, float* lse,
+                               unsigned flags, mla_stream_t stream);
 
 /* Read and clear the current device's status word: waits for `stream`, then
  * stores into *status the first error any kernel recorded since the last
