@@ -45,6 +45,26 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+def profiled_traffic(workload_name):
+    """DRAM bytes per decode launch from the committed ncu capture (profiles/traffic.json), or None
+    when the capture covers another workload or the kernel sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("workload") != workload_name:
+        return None
+    h = hashlib.sha256()
+    for rel in rec["source_files"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != rec["source_sha256_16"]:
+        return None
+    return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
+
+
 def workload_stats(w, lens):
     """Head-tokens, KV tokens, algorithmic bytes and flops of one decode."""
     s_q, H = w.s_q, w.H
@@ -363,6 +383,7 @@ def main():
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}
+    roof["traffic"] = profiled_traffic(w.name)
     roof["kernel"] = "mla_qdecode (decode kernel + split-KV combine, one C-ABI call)"
     roof["per_launch_ms"] = ms_decode
     roof["algorithmic"] = {"flops": st["flops"], "bytes": st["alg_bytes"]}
