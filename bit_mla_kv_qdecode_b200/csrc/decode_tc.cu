@@ -71,6 +71,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kCChunkStride = 1024;
 constexpr int kCLoOff = 512;
 constexpr int kCStage = kKChunks * kCChunkStride;
+constexpr int kBfChunkStride = 512;  // bf16 cache: C only, [chunk][token group][8 rows x 16 B]
 constexpr int kPTile = (kRows / 8) * 4 * 128;      // 8 KB: 16 row groups x 4 token groups x 128 B
 constexpr int kXRow = 36;                          // floats per row in the score-exchange buffer
 constexpr int kXBuf = kRows * kXRow * 4;
@@ -215,7 +216,11 @@ __device__ __forceinline__ void fail(const DecodeArgs& a, volatile int* abort_fl
   *abort_flag = 1;
 }
 
-template <int BITS_C, int G_C, int BITS_R, int G_R>
+// kBF16: the unquantized comparison cache (bf16 [pages][64][576]); the TMA
+// writes its rows straight into the operand layout (C_hi, no C_lo), the
+// "dequant" warps only zero rows past the end of the keys, scores need one
+// term and the output two (P_hi.C + P_lo.C). BITS_*/G_* are unused then.
+template <int BITS_C, int G_C, int BITS_R, int G_R, bool kBF16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TmapSet tm, int row_tiles, int n_terms_qk,
                      int n_terms_pv) {
@@ -309,7 +314,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // =========================== TMA producer ===========================
-    if (lane == 0) {
+    if (lane == 0 && kBF16) {
+      // bf16 rows land directly in operand stage j % kNC once PV of chunk j-kNC released it
+      int issued[kNC];
+      for (int i = 0; i < kNC; ++i) issued[i] = 0;
+      for (int j = 0; j < n_chunks; ++j) {
+        const int cs = j % kNC;
+        if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, kWaitLimitNs)) {
+          fail(a, abort_flag);
+          break;
+        }
+        const int t0 = t_begin + j * kChunk;
+        const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
+        uint8_t* st = smem + kOffC + cs * kCStage;
+        stage_page[cs] = page;
+        if (page >= 0) {
+          ptx::mbar_arrive_expect_tx(&bars.code_full[cs], kKChunks * kChunk * 16);
+          const int slot0 = t0 % kPage;
+          ptx::tma_load_4d(st, &tm.cc, 0, slot0, crank * (kHalfC / 8), page, &bars.code_full[cs]);
+          ptx::tma_load_4d(st + (kHalfC / 8) * kBfChunkStride, &tm.rc, 0, slot0, kDc / 8 + crank * (kHalfR / 8), page,
+                           &bars.code_full[cs]);
+        } else {
+          record_error(a.status, MLA_ERR_INVALID_ARG);
+          ptx::mbar_arrive(&bars.code_full[cs]);
+        }
+        issued[cs] = j + 1;
+      }
+      for (int cs = 0; cs < kNC; ++cs)
+        if (issued[cs] > 0) ptx::mbar_wait(&bars.code_full[cs], ((issued[cs] - 1) / kNC) & 1, nullptr, kWaitLimitNs);
+    } else if (lane == 0) {
       const uint32_t bytes = kChunk * (G::kRowC / 2) + kChunk * G::kRowR + kChunk * (G::kGroupsC * 2) +
                              kChunk * G::kGroupsR * 4;
       int issued[kNS];
@@ -355,8 +388,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const int par = (warp == 1) ? 0 : 1;
       uint64_t* drain = (warp == 1) ? bars.qk_drain : bars.qk_drain2;
-      const uint32_t idesc = ptx::idesc_bf16_f32(kRows, n_terms_qk == 2 ? 2 * kChunk : kChunk, 0, 0);
-      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), kCChunkStride, 128);
+      constexpr int cstride = kBF16 ? kBfChunkStride : kCChunkStride;
+      const uint32_t idesc = ptx::idesc_bf16_f32(kRows, (!kBF16 && n_terms_qk == 2) ? 2 * kChunk : kChunk, 0, 0);
+      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), cstride, 128);
       const uint64_t a_rope = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffQR), 128, 512);
       bool ok = ptx::mbar_wait(bars.q_full, 0, abort_flag, kWaitLimitNs);
       for (int j = par; ok && j < n_chunks; j += 2) {
@@ -371,12 +405,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t d = tmem + kTmemS + sb * 2 * kChunk;
 #pragma unroll
         for (int k = 0; k < kHalfC / 16; ++k)
-          ptx::mma_ts(d, tmem + kTmemQ + k * 8, bs + static_cast<uint64_t>((k * 2 * kCChunkStride) >> 4), idesc,
+          ptx::mma_ts(d, tmem + kTmemQ + k * 8, bs + static_cast<uint64_t>((k * 2 * cstride) >> 4), idesc,
                       k > 0 ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < kHalfR / 16; ++k)
           ptx::mma_ss(d, a_rope + static_cast<uint64_t>((k * 256) >> 4),
-                      bs + static_cast<uint64_t>(((kHalfC / 8 + 2 * k) * kCChunkStride) >> 4), idesc, 1u);
+                      bs + static_cast<uint64_t>(((kHalfC / 8 + 2 * k) * cstride) >> 4), idesc, 1u);
         ptx::mma_commit(&bars.s_full[sb]);
       }
       if (!ok) fail(a, abort_flag);
@@ -389,7 +423,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = ptx::idesc_bf16_f32(kRows, kHalfC, 0, 1);
       const uint64_t a0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffP), 128, 512);
-      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), 128, kCChunkStride);
+      const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), 128,
+                                                   kBF16 ? kBfChunkStride : kCChunkStride);
       bool ok = true;
       for (int j = 0; j < n_chunks; ++j) {
         const int pb = j & 1, cs = j % kNC;
@@ -420,7 +455,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int dq = tid - 64;
     const int tq = dq & 31;       // token within the chunk
     const int qsel = dq >> 5;     // 0..3
-    for (int j = 0; j < n_chunks; ++j) {
+    for (int j = 0; kBF16 && j < n_chunks; ++j) {
+      // bf16 operands are already in place; rows past the keys (stale pool
+      // rows, or a page the table could not name) are zeroed so that 0 * x
+      // never meets a NaN or Inf
+      const int cs = j % kNC;
+      if (!ptx::mbar_wait(&bars.code_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) { fail(a, abort_flag); break; }
+      const int t0 = t_begin + j * kChunk;
+      const int lim = stage_page[cs] >= 0 ? t_end - t0 : 0;
+      if (lim < kChunk && tq >= lim) {
+        uint8_t* st = smem + kOffC + cs * kCStage;
+#pragma unroll
+        for (int c = 0; c < kKChunks / 4; ++c)
+          *reinterpret_cast<uint4*>(st + (qsel * (kKChunks / 4) + c) * kBfChunkStride + tq * 16) = make_uint4(0, 0, 0, 0);
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(&bars.c_full[cs]);
+    }
+    for (int j = 0; !kBF16 && j < n_chunks; ++j) {
       const int s = j % kNS, cs = j % kNC;
       if (!ptx::mbar_wait(&bars.code_full[s], (j / kNS) & 1, abort_flag, kWaitLimitNs)) { fail(a, abort_flag); break; }
       if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, kWaitLimitNs)) {
@@ -766,44 +818,69 @@ bool make_map(CUtensorMap* m, const void* base, int width, int box_w, int page_b
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BC, int GC, int BR, int GR>
+// 4-D bf16 tensor [pages][64 tokens][72 chunks][8 channels] with the chunk
+// dimension outermost-but-one in shared memory: box = 8 channels x 32 tokens
+// x box_chunks x 1 page lands as [chunk][token][16 B], i.e. the no-swizzle
+// core-matrix layout with a 512-byte chunk stride.
+bool make_map_bf16(CUtensorMap* m, const void* base, int num_pages, int box_chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {8, static_cast<cuuint64_t>(kPage), static_cast<cuuint64_t>(kDqk / 8),
+                              static_cast<cuuint64_t>(num_pages)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(kDqk * 2), 16, static_cast<cuuint64_t>(kPage * kDqk * 2)};
+  const cuuint32_t box[4] = {8, static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(box_chunks), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BC, int GC, int BR, int GR, bool kBF16>
 cudaError_t launch_t(const DecodeLaunch& L) {
   using G = QGeom<BC, GC, BR, GR>;
   TmapSet tm;
   const uint8_t* pool = static_cast<const uint8_t*>(L.pool);
-  const CUtensorMapSwizzle swz_c = (BC == 4) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  if (!make_map(&tm.cc, pool + G::kOffCC, G::kRowC, G::kRowC / 2, G::kPageBytes, L.num_pages, swz_c) ||
-      !make_map(&tm.rc, pool + G::kOffRC, G::kRowR, G::kRowR, G::kPageBytes, L.num_pages,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&tm.cm, pool + G::kOffCM, G::kGroupsC * 4, G::kGroupsC * 2, G::kPageBytes, L.num_pages,
-                CU_TENSOR_MAP_SWIZZLE_NONE))
-    return cudaErrorNotSupported;
+  if constexpr (kBF16) {
+    if (!make_map_bf16(&tm.cc, pool, L.num_pages, kHalfC / 8) || !make_map_bf16(&tm.rc, pool, L.num_pages, kHalfR / 8))
+      return cudaErrorNotSupported;
+    tm.cm = tm.rc;
+  } else {
+    const CUtensorMapSwizzle swz_c = (BC == 4) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    if (!make_map(&tm.cc, pool + G::kOffCC, G::kRowC, G::kRowC / 2, G::kPageBytes, L.num_pages, swz_c) ||
+        !make_map(&tm.rc, pool + G::kOffRC, G::kRowR, G::kRowR, G::kPageBytes, L.num_pages,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tm.cm, pool + G::kOffCM, G::kGroupsC * 4, G::kGroupsC * 2, G::kPageBytes, L.num_pages,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorNotSupported;
+  }
   const DecodeArgs a = make_decode_args(L);
   const int row_tiles = (a.rows + kRows - 1) / kRows;
   const long units = static_cast<long>(a.B) * a.n_split * row_tiles;
   if (units * 2 > 0x7FFFFFFFL) return cudaErrorNotSupported;
-  auto kern = decode_tc_kernel<BC, GC, BR, GR>;
+  auto kern = decode_tc_kernel<BC, GC, BR, GR, kBF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;
   const bool fast = (L.flags & MLA_DECODE_FAST_UNCOMPENSATED) != 0;
-  kern<<<static_cast<unsigned>(units * 2), kThreads, kSmemAlloc, L.stream>>>(a, tm, row_tiles, fast ? 1 : 2,
-                                                                             fast ? 1 : 3);
+  const int terms_qk = (kBF16 || fast) ? 1 : 2;
+  const int terms_pv = fast ? 1 : (kBF16 ? 2 : 3);
+  kern<<<static_cast<unsigned>(units * 2), kThreads, kSmemAlloc, L.stream>>>(a, tm, row_tiles, terms_qk, terms_pv);
   return cudaGetLastError();
 }
 
 }  // namespace tc
 
 cudaError_t launch_decode_tc(const DecodeLaunch& L) {
-  if (!L.quantized || L.num_pages < 1) return cudaErrorNotSupported;
+  if (L.num_pages < 1) return cudaErrorNotSupported;
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess || major != 10 ||
       minor != 0)
     return cudaErrorNotSupported;
+  if (!L.quantized) return tc::launch_t<4, 64, 4, 64, true>(L);
 #define MLA_TC_CASE(BC, GC, BR, GR)                                              \
   if (L.bits_c == BC && L.group_c == GC && L.bits_r == BR && L.group_r == GR)  \
-    return tc::launch_t<BC, GC, BR, GR>(L);
+    return tc::launch_t<BC, GC, BR, GR, false>(L);
 #define MLA_TC_R(BC, GC) \
   MLA_TC_CASE(BC, GC, 4, 64) MLA_TC_CASE(BC, GC, 4, 32) MLA_TC_CASE(BC, GC, 2, 64) MLA_TC_CASE(BC, GC, 2, 32)
   MLA_TC_R(4, 64)
