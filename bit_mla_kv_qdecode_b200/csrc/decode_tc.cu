@@ -24,13 +24,15 @@
 // + P_hi*C_lo. All accumulation is fp32 in TMEM. This keeps the output within
 // 2e-3 of its RMS of the exact float64 result; single bf16 operands would not.
 //
-// Warp roles (384 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer: packed codes + metadata of 32-token chunks
 //   warp 1      TMEM owner; issues the QK MMAs of even chunks
 //   warp 6      issues the PV MMAs
 //   warp 7      issues the QK MMAs of odd chunks
 //   warps 2-5   unpack + dequantize into bf16 hi/lo operand tiles
-//   warps 8-11  one thread per row: score exchange, online softmax, P tiles,
+//   warps 8-15  two threads per row (warps w and w+4 share a TMEM lane
+//               quarter, 16 of each chunk's 32 columns each): score exchange,
+//               online softmax, P tiles,
 //               output rescaling in TMEM, epilogue
 // Every wait is bounded; a timeout sets MLA_ERR_TIMEOUT and the unit drains
 // and exits without touching memory it does not own.
@@ -46,7 +48,8 @@
 namespace mla {
 namespace tc {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kSoftThreads = 256;  // warps 8-15
 constexpr int kChunk = 32;            // tokens per pipeline step
 constexpr int kRows = 128;            // query rows per unit (MMA M)
 constexpr int kHalfC = 256;           // content channels per CTA
@@ -73,8 +76,13 @@ constexpr int kCLoOff = 512;
 constexpr int kCStage = kKChunks * kCChunkStride;
 constexpr int kBfChunkStride = 512;  // bf16 cache: C only, [chunk][token group][8 rows x 16 B]
 constexpr int kPTile = (kRows / 8) * 4 * 128;      // 8 KB: 16 row groups x 4 token groups x 128 B
-constexpr int kXRow = 36;                          // floats per row in the score-exchange buffer
-constexpr int kXBuf = kRows * kXRow * 4;
+// Score-exchange slot: [column half h][row][20 floats] (16 scores + 4 pad, a
+// bank-conflict-free stride for 16-byte accesses). The 32 rows one softmax warp
+// owns in one half are a contiguous 2560-byte block, sent as one bulk copy.
+constexpr int kXRowBytes = 80;
+constexpr int kXWarpBlock = 32 * kXRowBytes;
+constexpr int kXHalf = kRows * kXRowBytes;
+constexpr int kXBuf = 2 * kXHalf;
 constexpr int kCodeCC = 4096;                      // content codes half (32 tokens x <=128 B)
 constexpr int kCodeRC = 1024;                      // rope codes (32 tokens x <=32 B)
 constexpr int kCodeCM = 1024;                      // content meta half (32 tokens x <=32 B)
@@ -86,9 +94,10 @@ constexpr int kOffCode = kOffX + 2 * kXBuf;
 constexpr int kOffBar = kOffCode + kNS * kCodeStage + kRows * kHalfR * 2;
 constexpr int kOffQR = kOffCode + kNS * kCodeStage;  // rope part of Q: 128 rows x 32 bf16, core matrices
 constexpr int kQRBytes = kRows * kHalfR * 2;
-constexpr int kNumBars = 2 * kNS + 2 * kNC + 16;
+constexpr int kNumBars = 2 * kNS + 2 * kNC + 16 + 12;
 constexpr int kOffMisc = kOffQR + kQRBytes + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 64;
+constexpr int kOffRed = kOffMisc + 64;  // row-pair exchange: [2 parity][2 halves][128] maxima, [2][128] sums
+constexpr int kSmemBytes = kOffRed + (2 * 2 * kRows + 2 * kRows) * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;      // slack to align the base to 1024
 static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0, "TMA swizzle needs 1024-byte aligned stages");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -114,6 +123,8 @@ struct Bars {
   uint64_t* o_full;      // [1] all PV MMAs of the unit done
   uint64_t* qk_drain;    // [1] all QK MMAs of the even-chunk issuer done
   uint64_t* qk_drain2;   // [1] ... of the odd-chunk issuer
+  uint64_t* pair_max;    // [4 lane quarters][2 parity] both halves of a row published their chunk maximum
+  uint64_t* pair_sum;    // [4] both halves published their row sums (epilogue)
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
@@ -133,6 +144,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.o_full = p + 13;
   r.qk_drain = p + 14;
   r.qk_drain2 = p + 15;
+  r.pair_max = p + 16;
+  r.pair_sum = p + 24;
   return r;
 }
 
@@ -285,15 +298,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars.s_full[i], 1);
-      ptx::mbar_init(&bars.s_empty[i], 128);
-      ptx::mbar_init(&bars.p_full[i], 128);
+      ptx::mbar_init(&bars.s_empty[i], kSoftThreads);
+      ptx::mbar_init(&bars.p_full[i], kSoftThreads);
       ptx::mbar_init(&bars.p_empty[i], 1);
       ptx::mbar_init(&bars.x_full[i], 1);     // armed locally with expect_tx; bytes come from the peer
     }
-    ptx::mbar_init(bars.q_full, 128);
+    ptx::mbar_init(bars.q_full, kSoftThreads);
     ptx::mbar_init(bars.o_full, 1);
     ptx::mbar_init(bars.qk_drain, 1);
     ptx::mbar_init(bars.qk_drain2, 1);
+    for (int q = 0; q < 8; ++q) ptx::mbar_init(&bars.pair_max[q], 64);
+    for (int q = 0; q < 4; ++q) ptx::mbar_init(&bars.pair_sum[q], 64);
     *abort_flag = 0;
     ptx::fence_mbar_init_cluster();
   }
@@ -528,21 +543,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 8) {
     // =========================== softmax / epilogue ===========================
-    const int i = tid - 256;  // row within the tile == TMEM lane
+    // Two threads per row: warps w and w+4 read the same TMEM lane quarter;
+    // half h owns score columns [16h, 16h+16) of every chunk and output
+    // columns [128h, 128h+128) of this CTA's 256. The halves exchange their
+    // chunk maximum through shared memory (an mbarrier per lane quarter, so a
+    // stalled partner ends in a bounded wait), take identical softmax
+    // decisions, and add their partial row sums once, in the epilogue.
+    const int h = (warp - 8) >> 2;
+    const int quarter = warp & 3;
+    const int i = quarter * 32 + lane;  // row within the tile == TMEM lane
     const int row = row0 + i;
     const bool row_ok = row < a.rows;
     const int L = row_ok ? row_visible(T, a.s_q, a.H, row) : 0;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const size_t qrow = static_cast<size_t>(b) * a.rows + (row_ok ? row : 0);
+    float* red_max = reinterpret_cast<float*>(smem + kOffRed);   // [parity][half][row]
+    float* red_sum = red_max + 2 * 2 * kRows;                   // [half][row]
 
-    // Q: content half -> TMEM columns [384, 512); RoPE half -> shared memory
-    // (K-major core matrices, the A operand of the two RoPE K-steps).
-    // Padding rows get zeros.
+    // Q: content half -> TMEM columns [384, 512) (half h stores 64 of its 256
+    // channels' worth of columns); RoPE half -> shared memory as K-major core
+    // matrices (half h stores chunks 2h, 2h+1). Padding rows get zeros.
     {
       const uint4* qc = reinterpret_cast<const uint4*>(a.q_c + qrow * kDc + crank * kHalfC);
       const uint4* qr = reinterpret_cast<const uint4*>(a.q_r + qrow * kDr + crank * kHalfR);
 #pragma unroll
-      for (int blk = 0; blk < 4; ++blk) {
+      for (int bb = 0; bb < 2; ++bb) {
+        const int blk = 2 * h + bb;
         uint32_t v[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -553,28 +579,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       uint8_t* qrs = smem + kOffQR + (i >> 3) * 512 + (i & 7) * 16;
 #pragma unroll
-      for (int kc = 0; kc < 4; ++kc)
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * h + kk;
         *reinterpret_cast<uint4*>(qrs + kc * 128) = row_ok ? __ldg(qr + kc) : make_uint4(0, 0, 0, 0);
+      }
       ptx::fence_proxy_async_smem();
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(bars.q_full);
     }
 
-    // Score exchange. Step j first finishes chunk j-1 (its peer half arrived
-    // during the previous step), then reads this CTA's partial S_j from TMEM
-    // and stores it into the peer's exchange buffer with st.async, which
-    // completes bytes on the peer's x_full. Two buffers suffice without any
-    // release handshake: the peer sends chunk j-1 only after it has read
-    // chunk j-2, and this thread sees chunk j-1 arrive before it sends chunk j
-    // into the buffer chunk j-2 used.
+    // Score exchange. Step j first finishes chunk j-1 (its peer partial was
+    // sent at the end of the previous step), then reads this CTA's partial
+    // S_j from TMEM, stages it in the exchange slot it has just read, and
+    // each warp bulk-copies its 32 rows x 16 columns to the same place in the
+    // peer's slot j&1 (the copy engine completes the bytes on the peer's
+    // x_full). No release handshake is needed: the peer sends chunk j+1 into
+    // the staging slot only after it received chunk j, i.e. after this
+    // copy has read the stage.
     const uint32_t xbuf_peer = ptx::mapa(ptx::smem_u32(smem + kOffX), peer);
     const uint32_t xfull_peer = ptx::mapa(ptx::smem_u32(bars.x_full), peer);
-    float m_used = -CUDART_INF_F, l_sum = 0.0f;
+    float m_used = -CUDART_INF_F, l_sum = 0.0f;  // l_sum: this half's columns only
     bool o_live = false;  // O has been written by a PV MMA
     bool ok = true;
-    uint32_t prev[32];
-    bool prev_page_ok = false;
+    uint32_t prev[16];
+    int prev_page = -1;
 
     for (int j = 0; j <= n_chunks && ok; ++j) {
       if (j >= 1) {
@@ -584,12 +613,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + pb * kXBuf + i * (kXRow * 4));
+        const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + pb * kXBuf + h * kXHalf + i * kXRowBytes);
         // full score = my partial + peer partial, then * scale * log2(e)
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-        float2 sp[16];
+        float2 sp[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
           const float4 pv = xr[k];
           sp[2 * k] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k]), __uint_as_float(prev[4 * k + 1])),
                                             make_float2(pv.x, pv.y)), sc2);
@@ -597,22 +626,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                             __uint_as_float(prev[4 * k + 3])),
                                                 make_float2(pv.z, pv.w)), sc2);
         }
-        const int lim = prev_page_ok ? min(L, t_end) - t0 : 0;
-        if (lim < kChunk) {  // partially visible chunk (ragged tail, causal row, bad page)
+        const int lim = (page_valid(prev_page, a.num_pages) ? min(L, t_end) - t0 : 0) - 16 * h;  // visible columns in my half
+        if (lim < 16) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             if (2 * k >= lim) sp[k].x = -CUDART_INF_F;
             if (2 * k + 1 >= lim) sp[k].y = -CUDART_INF_F;
           }
         }
-        float mt[16];
+        float mt[8];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) mt[k] = fmaxf(sp[k].x, sp[k].y);
+        for (int k = 0; k < 8; ++k) mt[k] = fmaxf(sp[k].x, sp[k].y);
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
+        for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
           for (int k = 0; k < w; ++k) mt[k] = fmaxf(mt[k], mt[k + w]);
-        const float mx = mt[0];
+        // chunk maximum of the whole row: publish mine, wait for the other half's
+        red_max[(pb * 2 + h) * kRows + i] = mt[0];
+        ptx::mbar_arrive(&bars.pair_max[quarter * 2 + pb]);
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.pair_max[quarter * 2 + pb], (jj >> 1) & 1, abort_flag,
+                                              kWaitLimitNs))) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(mt[0], red_max[(pb * 2 + (h ^ 1)) * kRows + i]);
         float alpha = 1.0f;
         bool rescale = false;
         if (mx > -CUDART_INF_F) {
@@ -627,10 +664,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // p = 2^(s - m); rows that have seen no key use m = 0, so every p is 0
         const float m_eff = (m_used == -CUDART_INF_F) ? 0.0f : m_used;
         const float2 negm = make_float2(-m_eff, -m_eff);
-        uint32_t ph[16], pl[16];
-        float2 ps[16];
+        uint32_t ph[8], pl[8];
+        float2 ps[8];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
+        for (int k = 0; k < 8; ++k) {
           const float2 d = __fadd2_rn(sp[k], negm);
           const float2 pk = make_float2(ex2_approx(d.x), ex2_approx(d.y));
           ps[k] = pk;
@@ -642,13 +679,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           pl[k] = *reinterpret_cast<uint32_t*>(&lb);
         }
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
+        for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
           for (int k = 0; k < w; ++k) ps[k] = __fadd2_rn(ps[k], ps[k + w]);
-        const float psum = ps[0].x + ps[0].y;
-        l_sum = l_sum * alpha + psum;
+        l_sum = l_sum * alpha + (ps[0].x + ps[0].y);
 
-        // P tile (this row) -> smem, once PV of chunk jj-2 released the buffer
+        // P tile (my 16 tokens of this row) -> smem, once PV of chunk jj-2 released the buffer
         if (jj >= 2 &&
             !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
           ok = false;
@@ -656,15 +692,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
 #pragma unroll
-        for (int kc = 0; kc < 4; ++kc) {
+        for (int kk = 0; kk < 2; ++kk) {
+          const int kc = 2 * h + kk;
           *reinterpret_cast<uint4*>(pt + kc * 128) =
-              make_uint4(ph[4 * kc], ph[4 * kc + 1], ph[4 * kc + 2], ph[4 * kc + 3]);
+              make_uint4(ph[4 * kk], ph[4 * kk + 1], ph[4 * kk + 2], ph[4 * kk + 3]);
           *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
-              make_uint4(pl[4 * kc], pl[4 * kc + 1], pl[4 * kc + 2], pl[4 * kc + 3]);
+              make_uint4(pl[4 * kk], pl[4 * kk + 1], pl[4 * kk + 2], pl[4 * kk + 3]);
         }
 
-        // rescale this row's half of O in TMEM (warp-collective: lanes that do
-        // not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
+        // rescale my half of this row of O in TMEM (warp-collective: lanes that
+        // do not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
         if (__any_sync(kFull, rescale && o_live)) {
           if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
                                                 kWaitLimitNs))) {
@@ -674,13 +711,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
           const float f = (rescale && o_live) ? alpha : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < kHalfC / 32; ++c) {
+          for (int c = 0; c < kHalfC / 64; ++c) {
             uint32_t ov[32];
-            ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+            ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
             ptx::tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            ptx::tmem_st32(lane_base + kTmemO + c * 32, ov);
+            ptx::tmem_st32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
           }
           ptx::tmem_st_wait();
         }
@@ -689,56 +726,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars.p_full[pb]);
       }
-      uint32_t cur[32];
-      bool cur_page_ok = false;
+      uint32_t cur[16];
+      int cur_page = -1;
       if (j < n_chunks) {
         const int sb = j & 1;
+        // block-table entry of chunk j, checked one step later: issued before the wait to hide the load
+        cur_page = table_entry(a.table, a.max_pages, b, t_begin + j * kChunk);
         // wait results are made warp-uniform: the TMEM loads below are warp-collective
         if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        ptx::tmem_ld32(lane_base + kTmemS + sb * 2 * kChunk, cur);
+        ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + 16 * h, cur);
         if (n_terms_qk == 2) {  // add the C_lo half of the score tile
-          uint32_t lo[32];
-          ptx::tmem_ld32(lane_base + kTmemS + sb * 2 * kChunk + kChunk, lo);
+          uint32_t lo[16];
+          ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + kChunk + 16 * h, lo);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) cur[k] = __float_as_uint(__uint_as_float(cur[k]) + __uint_as_float(lo[k]));
+          for (int k = 0; k < 16; ++k) cur[k] = __float_as_uint(__uint_as_float(cur[k]) + __uint_as_float(lo[k]));
         }
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars.s_empty[sb]);
-        // page validity of chunk j, consumed one step later (hides the load)
-        cur_page_ok = lookup_page(a.table, a.max_pages, a.num_pages, b, t_begin + j * kChunk) >= 0;
-        if (i == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kRows * kChunk * 4);
-        const uint32_t dst = xbuf_peer + sb * kXBuf + i * (kXRow * 4);
+        // Send my partial scores to the peer. They are staged in the other
+        // exchange slot, whose segment for my row and half I finished reading
+        // above (chunk j-1); the peer writes that slot again (chunk j+1) only
+        // after this copy has landed, and I restage it only after that.
+        const int blk = h * kXHalf + quarter * kXWarpBlock;
+        uint8_t* stage = smem + kOffX + (sb ^ 1) * kXBuf + h * kXHalf + i * kXRowBytes;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          ptx::st_async_v4(dst + k * 16, cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3],
-                           xfull_peer + sb * 8);
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(stage + 16 * k) = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (i == 0 && h == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kXBuf);
+        if (lane == 0)
+          ptx::bulk_copy_to_peer(xbuf_peer + sb * kXBuf + blk, smem + kOffX + (sb ^ 1) * kXBuf + blk, kXWarpBlock,
+                                 xfull_peer + sb * 8);
       }
 #pragma unroll
-      for (int k = 0; k < 32; ++k) prev[k] = cur[k];
-      prev_page_ok = cur_page_ok;
+      for (int k = 0; k < 16; ++k) prev[k] = cur[k];
+      prev_page = cur_page;
     }
 
-    // epilogue: O / l for this CTA's 256 channels
+    // epilogue: row sum = both halves; O / l for my 128 of this CTA's 256 channels
     if (!ok) fail(a, abort_flag);
+    red_sum[h * kRows + i] = l_sum;
+    ptx::mbar_arrive(&bars.pair_sum[quarter]);
+    const bool sums_ready = ptx::mbar_wait(&bars.pair_sum[quarter], 0, abort_flag, kWaitLimitNs);
     const bool o_ready = ptx::mbar_wait(bars.o_full, 0, abort_flag, kWaitLimitNs);
     const int aborted = *abort_flag;
-    if (__all_sync(kFull, o_ready && ok && !aborted)) {  // warp-uniform: TMEM loads are collective
+    if (__all_sync(kFull, sums_ready && o_ready && ok && !aborted)) {  // warp-uniform: TMEM loads are collective
       ptx::tc_fence_after();
-      const float inv = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
-      const float lse = l_sum > 0.0f ? (m_used + log2f(l_sum)) * kLn2 : -CUDART_INF_F;
+      const float l_tot = l_sum + red_sum[(h ^ 1) * kRows + i];
+      const float inv = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
+      const float lse = l_tot > 0.0f ? (m_used + log2f(l_tot)) * kLn2 : -CUDART_INF_F;
       const size_t part = (static_cast<size_t>(b) * a.n_split + split) * a.rows + row;
 #pragma unroll 1
-      for (int c = 0; c < kHalfC / 32; ++c) {
+      for (int c = 0; c < kHalfC / 64; ++c) {
         uint32_t ov[32];
-        ptx::tmem_ld32(lane_base + kTmemO + c * 32, ov);
+        ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
         ptx::tmem_ld_wait();
-        const int col = crank * kHalfC + c * 32;
+        const int col = crank * kHalfC + h * (kHalfC / 2) + c * 32;
         if (!row_ok) continue;
         if (a.n_split == 1 && !a.out_f32) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc + col);
@@ -747,9 +797,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(ov[8 * k + 2 * e]) * inv,
-                                                       __uint_as_float(ov[8 * k + 2 * e + 1]) * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&h);
+              __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(ov[8 * k + 2 * e]) * inv,
+                                                        __uint_as_float(ov[8 * k + 2 * e + 1]) * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&hv);
             }
             dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
           }
@@ -763,7 +813,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                  __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
         }
       }
-      if (crank == 0 && row_ok) {
+      if (crank == 0 && h == 0 && row_ok) {
         if (a.n_split == 1) {
           if (a.lse) a.lse[qrow] = lse;
         } else {
@@ -780,7 +830,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmemCols);
   }
-  ptx::cluster_sync();  // no remote store or arrive may target a CTA that has exited
+  // No remote copy or arrive may target a CTA that has exited. After a clean
+  // run every score copy has landed (each one was waited for); after an abort
+  // one may still be in flight, so give it time to land before either exits.
+  ptx::cluster_sync();
+  if (tid == 0 && (*abort_flag || ptx::ld_cluster_s32(ptx::mapa(ptx::smem_u32((const void*)abort_flag), peer)))) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (ptx::globaltimer_ns() - t0 < 100000ull) {
+    }
+  }
+  ptx::cluster_sync();
 }
 
 // ---------------------------------------------------------------- host side

@@ -52,12 +52,20 @@ __device__ __forceinline__ float half_bits_to_float(uint32_t h) {
 
 // Page of token position t of request b, or -1 when the position or table
 // entry is out of range (the caller skips such tokens and flags the status).
-__device__ __forceinline__ int lookup_page(const int32_t* table, int max_pages, int num_pages,
-                                           int b, int t) {
+// The block-table entry for token t, not yet checked against the pool (-1 past
+// the table's end): a caller can issue the load early and validate where it uses it.
+__device__ __forceinline__ int table_entry(const int32_t* table, int max_pages, int b, int t) {
   int idx = t / kPage;
   if (t < 0 || idx >= max_pages) return -1;
-  int page = __ldg(table + static_cast<size_t>(b) * max_pages + idx);
-  return (page >= 0 && page < num_pages) ? page : -1;
+  return __ldg(table + static_cast<size_t>(b) * max_pages + idx);
+}
+
+__device__ __forceinline__ bool page_valid(int page, int num_pages) { return page >= 0 && page < num_pages; }
+
+__device__ __forceinline__ int lookup_page(const int32_t* table, int max_pages, int num_pages,
+                                           int b, int t) {
+  const int page = table_entry(table, max_pages, b, t);
+  return page_valid(page, num_pages) ? page : -1;
 }
 
 // Arguments shared by the decode kernels.
