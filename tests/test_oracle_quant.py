@@ -167,3 +167,29 @@ def test_page_writer_offsets_and_reader():
     assert np.array_equal(C, quant.dequantize_groups(u, s, z, 32))
     u, s, z = quant.quantize_groups(r[0], 4, 64)
     assert np.array_equal(R, quant.dequantize_groups(u, s, z, 64))
+
+
+def test_batched_append_uses_each_requests_table():
+    # Layout rule: token t of request b lives in page block_table[b][t // P],
+    # slot t % P. One append call for two requests with different histories:
+    # request 1's new tokens must land in its own pages (byte check at a
+    # hand-computed offset), and request 0's pages must hold only its tokens.
+    desc = layout.Desc()
+    rng = np.random.default_rng(11)
+    c = (rng.standard_normal((2, 3, 512)).astype(np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)
+    r = (rng.standard_normal((2, 3, 64)).astype(np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)
+    table = np.array([[1, 3], [2, 0]], dtype=np.int32)
+    pool = layout.new_pool(desc, 4)
+    layout.append(desc, pool, table, [62, 5], c, r)
+    # request 1, new token 0 is t = 5 -> page table[1][0] = 2, slot 5
+    uc, _, _ = quant.quantize_groups(c[1, 0:1], 4, 64)
+    assert np.array_equal(pool[2, 5 * 256:6 * 256], quant.pack_codes(uc, 4)[0])
+    # request 0, new token 2 is t = 64 -> page table[0][1] = 3, slot 0
+    uc, _, _ = quant.quantize_groups(c[0, 2:3], 4, 64)
+    assert np.array_equal(pool[3, 0:256], quant.pack_codes(uc, 4)[0])
+    # page 0 (request 1's second page) is untouched
+    assert not pool[0].any()
+    for b, t0 in ((0, 62), (1, 5)):
+        C, _ = layout.gather_tokens(desc, pool, table[b], t0 + 3)
+        u, s, z = quant.quantize_groups(c[b], 4, 64)
+        assert np.array_equal(C[t0:t0 + 3], quant.dequantize_groups(u, s, z, 64))
