@@ -65,6 +65,19 @@ def profiled_traffic(workload_name):
     return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
 
 
+def max_over_ranks(x, dist, device):
+    """The largest of every rank's x: a multi-rank job ends when its slowest rank does."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: every rank runs the same workload (weak scaling), all within ms."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 def workload_stats(w, lens):
     """Head-tokens, KV tokens, algorithmic bytes and flops of one decode."""
     s_q, H = w.s_q, w.H
@@ -360,9 +373,7 @@ def main():
         torch.cuda.synchronize()
     ms_total = t_start.elapsed_time(t_end)
     if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+        ms_total = max_over_ranks(ms_total, dist, dev)
         dist.barrier()
     ms_step = ms_total / args.steps
     ms_append = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(args.steps))
@@ -370,7 +381,7 @@ def main():
     assert api.mla_get_device_status() == 0
 
     st = workload_stats(w, lens)
-    value = st["head_tokens"] * world / (ms_step * 1e-3)
+    value = job_rate(st["head_tokens"], world, ms_step)
     peaks, peak_src = load_peaks()
     flop_rate = st["flops"] / (ms_decode * 1e-3) / 1e12
     gbs = st["alg_bytes"] / (ms_decode * 1e-3) / 1e9
@@ -443,9 +454,7 @@ def main():
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / args.steps
     if world > 1:
-        tt = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
+        ms_e2e = max_over_ranks(ms_e2e, dist, dev)
     h2d = (h_qc.numel() + h_qr.numel() + h_nc.numel() + h_nr.numel()) * 2
     d2h = h_out.numel() * 2 + h_lse.numel() * 4
 
@@ -455,12 +464,12 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 hi+lo operand pairs, f32 accumulate", "data": "synthetic",
         "config": _config(w, world, extra={"num_splits": n_split, "pool_copies": R, "pool_mb": pool_bytes / 1e6}),
-        "kv_tokens_per_s": st["kv_tokens"] * world / (ms_step * 1e-3),
+        "kv_tokens_per_s": job_rate(st["kv_tokens"], world, ms_step),
         "hbm": {"achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
                 "note": "algorithmic bytes of one decode / decode-call time"},
         "legs_ms": {"append": ms_append, "decode": ms_decode},
         "roofline": roof,
-        "e2e": {"value": st["head_tokens"] * world / (ms_e2e * 1e-3), "unit": "head-tokens/s",
+        "e2e": {"value": job_rate(st["head_tokens"], world, ms_e2e), "unit": "head-tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches_per_step * args.steps,
         "bf16_decode": bf16_leg,
