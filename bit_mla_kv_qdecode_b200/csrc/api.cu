@@ -60,16 +60,18 @@ struct SplitPlan {
 // is honoured (capped at the page count). The automatic choice models the
 // decode time of the longest request as waves(n) * (pages / n), where a wave
 // is one work unit (128 query rows of one request and one split) on each
-// 2-CTA cluster slot, and picks the smallest n within 3% of the best, with
-// chunks of at least 4 pages.
+// 2-CTA cluster slot -- or, for at most 16 query rows, one request and split
+// on each of two CTA slots per SM (the small-row kernel) -- and picks the
+// smallest n within 3% of the best, with chunks of at least 4 pages.
 SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
   const int pages = std::max(1, (max_seq_len + mla::kPage - 1) / mla::kPage);
   int n;
   if (requested > 0) {
     n = std::min(requested, pages);
   } else {
-    const long units = static_cast<long>(std::max(B, 1)) * ((static_cast<long>(s_q) * H + 127) / 128);
-    const long slots = std::max(1, device_sm_count() / 2);
+    const bool small = static_cast<long>(s_q) * H <= mla::kSmallRows;
+    const long units = static_cast<long>(std::max(B, 1)) * (small ? 1 : (static_cast<long>(s_q) * H + 127) / 128);
+    const long slots = std::max(1, small ? 2 * device_sm_count() : device_sm_count() / 2);
     const int n_max = std::max(1, std::min(pages / 4, 64));
     double best = 1e30;
     n = 1;
@@ -176,7 +178,13 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   L.stream = c.stream;
 
   cudaError_t e = cudaErrorNotSupported;
-  if (!(c.flags & MLA_DECODE_FORCE_SIMT)) e = mla::launch_decode_tc(L);
+  if (!(c.flags & MLA_DECODE_FORCE_SIMT)) {
+    e = mla::launch_decode_small(L);
+    if (e == cudaErrorNotSupported) {
+      cudaGetLastError();
+      e = mla::launch_decode_tc(L);
+    }
+  }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
     e = mla::launch_decode_simt(L);

@@ -1,0 +1,505 @@
+// Decode for few query rows (s_q * H <= 16) on warp-level tensor-core MMAs
+// (mma.sync m16n8k16). With 16 rows a 128-row tcgen05 tile would be 7/8
+// padding, so this kernel keeps the rows at the MMA's native M = 16 and lets
+// the tokens carry the N and K dimensions.
+//
+// Absorbed MQA decode over the low-bit latent cache: scores
+// (q_c . c_hat_t + q_r . kr_hat_t) * scale, softmax, output sum_t p_t c_hat_t
+// (Group-Query Latent Attention abstract: one absorbed decoding path over the
+// shared latent; QuantMLA abstract: dequantization inside the attention).
+//
+// Scores are exact in the codes. For a 64-channel group with scale s and
+// zero z, q . c_hat = s * (q . (u + 128)) + (z - 128 s) * sum(q): the MMA takes
+// the integer codes as bf16 values u + 128 (exact, built by a byte permute),
+// q is bf16, products are exact and accumulate in fp32; s and z are applied
+// per (token, group) in fp32 afterwards. The output is exact in the codes as
+// well: for a group, sum_t p_t c_hat_t = sum_t (p_t s_t) u_t + sum_t p_t z_t.
+// The MMA takes the codes as the exact fp16 values u * 2^-24 (the subnormal
+// whose bits are [u, 0x00]) and the weights w_t = p_t s_t as an fp16 hi + lo
+// pair (22 significant bits, two MMAs); the epilogue scales by 2^24 and adds
+// sum_t p_t z_t, accumulated in fp32 per (row, group).
+//
+// One CTA per (request, split): whole 64-token pages are bulk-copied into a
+// 4-stage ring (issued by one thread, three pages ahead); eight warps split each page's tokens for
+// the scores (8 keys each) and its channels for the output (one 64-channel
+// group each, the accumulators stay in registers). One named barrier per page hands the
+// weights and per-warp maxima across; the running maximum is lazy (it moves
+// only when a score exceeds it by more than 2^8), so the common page needs no
+// rescale.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <math_constants.h>
+
+#include "mla_common.cuh"
+#include "mla_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace small {
+
+constexpr int kWarps = 8;                    // compute warps
+constexpr int kThreads = 32 * kWarps;
+constexpr int kNS = 4;                       // page stages
+constexpr int kRows = 16;                    // MMA M
+constexpr int kGroups = 9;                   // 8 content groups of 64 + the RoPE group of 64
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kPRow = (kPage + 8) * 4;       // weight tile row stride (bytes): 64 fp32 + pad
+constexpr int kPTile = kRows * kPRow;
+constexpr int kORow = kDc + 4;               // epilogue output tile row stride (floats)
+constexpr float kCodeScale = 16777216.0f;    // 2^24: the output MMA sees the codes as u * 2^-24
+
+template <class G>
+struct Layout {
+  static constexpr int kStage = (G::kPageBytes + 127) / 128 * 128;
+  static constexpr int kOffQ = kNS * kStage;                  // Q A-fragments [group][k-step][lane] x 16 B
+  static constexpr int kOffQSum = kOffQ + kGroups * 4 * 32 * 16;  // [group][row] float
+  static constexpr int kOffP = kOffQSum + kGroups * kRows * 4;    // [2][16 rows][kPRow] fp32 weights
+  static constexpr int kOffM = kOffP + 2 * kPTile;                // [2][16 rows][4 warps] float maxima
+  static constexpr int kOffL = kOffM + 2 * kRows * kWarps * 4;    // [16 rows][4 warps] float row sums
+  static constexpr int kOffBar = kOffL + kRows * kWarps * 4;      // full[kNS]
+  static constexpr int kOffMisc = kOffBar + kNS * 8;              // abort flag, stage page ids
+  static constexpr int kBytes = kOffMisc + 64;
+  static_assert(kRows * kORow * 4 <= kNS * kStage, "epilogue tile reuses the page stages");
+  static_assert(kOffQ % 16 == 0 && kOffP % 16 == 0 && kOffM % 16 == 0 && kOffBar % 8 == 0, "alignment");
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Byte j of a -> byte 0, byte j of b -> byte 2; bytes 1 and 3 replicate the
+// sign bit of those bytes, which is 0 for the nibble-per-byte inputs used here.
+__host__ __device__ constexpr uint32_t sel_pair(int j) {
+  return static_cast<uint32_t>(j | ((8 | j) << 4) | ((4 + j) << 8) | ((12 + j) << 12));
+}
+
+// Four 16-bit operand pairs from two nibble-per-byte words a, b (values
+// 0..15 in the low half of each byte): pair j = (a.byte j, b.byte j), each
+// completed with the high byte hb (0x43: bf16 128 + u; 0x64: fp16 1024 + u).
+// Three byte permutes per two pairs: interleave first, then merge the constant.
+__device__ __forceinline__ void nibble_pairs(uint32_t a, uint32_t b, uint32_t hb4, uint32_t (&p)[4]) {
+  const uint32_t m01 = prmt(a, b, 0x5140u), m23 = prmt(a, b, 0x7362u);  // [a0 b0 a1 b1], [a2 b2 a3 b3]
+  p[0] = prmt(m01, hb4, 0x4140u);  // [a0, hb, b0, hb]
+  p[1] = prmt(m01, hb4, 0x4342u);  // [a1, hb, b1, hb]
+  p[2] = prmt(m23, hb4, 0x4140u);
+  p[3] = prmt(m23, hb4, 0x4342u);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void named_barrier_compute() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// fp16 hi + lo of two fp32 values (hi = RN(x), lo = RN(x - hi)).
+__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  hi = h2_bits(h);
+  lo = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+}
+
+template <int BITS_C, int G_C, int BITS_R, int G_R>
+__global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeArgs a) {
+  using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
+  using Lo = Layout<G>;
+  static_assert(BITS_C == 4 && G_C == 64 && BITS_R == 4 && G_R == 64, "INT4 g64 content and RoPE");
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lo::kOffBar);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lo::kOffMisc);
+  volatile int* stage_page = reinterpret_cast<volatile int*>(smem + Lo::kOffMisc + 16);  // [kNS]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x / a.n_split;
+  const int split = blockIdx.x % a.n_split;
+  const int T = checked_len(a, b);
+  const int pages_b = (T + kPage - 1) / kPage;
+  const int p_begin = split * a.chunk_pages;
+  const int p_end = min(pages_b, p_begin + a.chunk_pages);
+  const int n_pages = max(0, p_end - p_begin);
+  const int t_end = min(T, p_end * kPage);  // keys this unit may see
+  if (a.n_split > 1 && p_begin >= pages_b) return;  // split past the last page: never read by the merge
+
+  if (tid == 0) {
+    for (int s = 0; s < kNS; ++s) ptx::mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init_cluster();
+  }
+  __syncthreads();
+
+  // Page k of the unit goes to stage k % kNS. Thread 0 issues pages
+  // 0 .. kNS-2 here and page k + kNS - 1 right after page k's named barrier,
+  // when every warp is past the output MMAs of page k - 1, the last reader of
+  // that stage. A missing page arrives without bytes; its keys are masked.
+  int n_issued = 0;
+  auto issue_page = [&](int k) {
+    if (k >= n_pages) return;
+    const int s = k % kNS;
+    const int page = table_entry(a.table, a.max_pages, b, (p_begin + k) * kPage);
+    if (page_valid(page, a.num_pages)) {
+      stage_page[s] = page;
+      ptx::mbar_arrive_expect_tx(&full[s], G::kPageBytes);
+      ptx::bulk_load(smem + s * Lo::kStage, a.pool + static_cast<size_t>(page) * G::kPageBytes, G::kPageBytes,
+                     &full[s]);
+    } else {
+      stage_page[s] = -1;
+      ptx::mbar_arrive(&full[s]);
+    }
+    n_issued = k + 1;
+  };
+  if (tid == 0)
+    for (int k = 0; k < kNS - 1; ++k) issue_page(k);
+
+  {
+    // =========================== compute warps ===========================
+    const int w = warp;
+    const int r = lane >> 2, kp = lane & 3;  // MMA fragment coordinates: row group, k pair
+    const bool row_ok0 = r < a.rows, row_ok1 = r + 8 < a.rows;
+    const int lim0 = row_ok0 ? min(row_visible(T, a.s_q, a.H, r), t_end) : 0;
+    const int lim1 = row_ok1 ? min(row_visible(T, a.s_q, a.H, r + 8), t_end) : 0;
+
+    // Q as A fragments, one 16-byte entry per (group, k-step, lane). Within a
+    // 64-channel group, K-step s pairs logical columns {2kp, 2kp+1} with
+    // channels 16kp + 4s + {0,1} and {8+2kp, 9+2kp} with 16kp + 4s + {2,3}:
+    // the code bytes one lane needs for all four K-steps are then the 8
+    // contiguous bytes [8kp, 8kp+8) of the token's group.
+    {
+      const uint32_t* qc = reinterpret_cast<const uint32_t*>(a.q_c);
+      const uint32_t* qr = reinterpret_cast<const uint32_t*>(a.q_r);
+      uint4* qf = reinterpret_cast<uint4*>(smem + Lo::kOffQ);
+      for (int e = tid; e < kGroups * 4 * 32; e += kWarps * 32) {
+        const int g = e / 128, s = (e / 32) & 3, ln = e & 31;
+        const int er = ln >> 2, ekp = ln & 3;
+        const int c = 16 * ekp + 4 * s;  // channel within the group
+        const bool ok0 = er < a.rows, ok1 = er + 8 < a.rows;
+        const size_t q0 = static_cast<size_t>(b) * a.rows + er, q1 = q0 + 8;
+        auto ld = [&](bool ok, size_t q, int cc) -> uint32_t {
+          if (!ok) return 0u;
+          return g < 8 ? __ldg(qc + (q * kDc + 64 * g + cc) / 2) : __ldg(qr + (q * kDr + cc) / 2);
+        };
+        qf[e] = make_uint4(ld(ok0, q0, c), ld(ok1, q1, c), ld(ok0, q0, c + 2), ld(ok1, q1, c + 2));
+      }
+      // per (group, row) sums of q, for the zero-point and code-offset term
+      float* qsum = reinterpret_cast<float*>(smem + Lo::kOffQSum);
+      for (int e = tid; e < kGroups * kRows; e += kWarps * 32) {
+        const int g = e / kRows, row = e % kRows;
+        float acc = 0.0f;
+        if (row < a.rows) {
+          const __nv_bfloat16* q = (g < 8) ? a.q_c + (static_cast<size_t>(b) * a.rows + row) * kDc + 64 * g
+                                           : a.q_r + (static_cast<size_t>(b) * a.rows + row) * kDr;
+          for (int c = 0; c < 64; ++c) acc += __bfloat162float(q[c]);
+        }
+        qsum[e] = acc;
+      }
+      named_barrier_compute();
+    }
+    const uint4* qfrag = reinterpret_cast<const uint4*>(smem + Lo::kOffQ);
+    const float* qsum = reinterpret_cast<const float*>(smem + Lo::kOffQSum);
+    float o[8][4];  // output accumulators of group w: block j, fragment c (see the epilogue)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+    float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};  // running maximum (log2 units) of rows r, r+8
+    float l_acc[2] = {0.0f, 0.0f};                      // this thread's share of the row sums, scaled to m_run
+    float corr[2] = {0.0f, 0.0f};                       // this thread's share of sum p z of group w, rows r, r+8
+    const float sl2 = a.scale_log2;
+
+    for (int k = 0; k < n_pages; ++k) {
+      const int s = k % kNS, pb = k & 1;
+      // on a timeout the loop runs on (every warp keeps the same barrier
+      // sequence) with the abort flag set, so later waits return at once
+      if (!ptx::mbar_wait(&full[s], (k / kNS) & 1, abort_flag, kWaitLimitNs)) {
+        record_error(a.status, MLA_ERR_TIMEOUT);
+        *abort_flag = 1;
+      }
+      const uint8_t* st = smem + s * Lo::kStage;
+      const bool page_ok = stage_page[s] >= 0;
+      const int P0 = (p_begin + k) * kPage;  // first key of the page
+
+      // ---- scores of this warp's 8 keys (one n-tile): lane (r, kp) feeds key 8w + r ----
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int tlb = 8 * w + r;       // key of this lane's B column
+      const int tl0 = 8 * w + 2 * kp;  // keys of this lane's accumulator columns: tl0, tl0 + 1
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) {
+        const uint2 cw = *reinterpret_cast<const uint2*>(
+            st + (g < 8 ? G::kOffCC + tlb * G::kRowC + 32 * g : G::kOffRC + tlb * G::kRowR) + 8 * kp);
+        // code byte i of the lane's 8 -> bf16 pair (128 + u_even, 128 + u_odd); K-step ks uses bytes 2ks, 2ks+1
+        uint32_t bq[2][4];
+        nibble_pairs(cw.x & 0x0F0F0F0Fu, (cw.x >> 4) & 0x0F0F0F0Fu, 0x43434343u, bq[0]);
+        nibble_pairs(cw.y & 0x0F0F0F0Fu, (cw.y >> 4) & 0x0F0F0F0Fu, 0x43434343u, bq[1]);
+        float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint4 af = qfrag[(g * 4 + ks) * 32 + lane];
+          mma_bf16(d, af, bq[ks >> 1][2 * (ks & 1)], bq[ks >> 1][2 * (ks & 1) + 1]);
+        }
+        // s * D + (z - 128 s) * sum(q) for this lane's two keys
+        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(
+            st + (g < 8 ? G::kOffCM + tl0 * G::kGroupsC * 4 + 4 * g : G::kOffRM + tl0 * 4));
+        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(
+            st + (g < 8 ? G::kOffCM + (tl0 + 1) * G::kGroupsC * 4 + 4 * g : G::kOffRM + (tl0 + 1) * 4));
+        const float2 sz0 = __half22float2(bits_h2(m0)), sz1 = __half22float2(bits_h2(m1));  // (s, z)
+        const float e0 = fmaf(-128.0f, sz0.x, sz0.y), e1 = fmaf(-128.0f, sz1.x, sz1.y);
+        const float qa = qsum[g * kRows + r], qb = qsum[g * kRows + r + 8];
+        sc[0] = fmaf(sz0.x, d[0], fmaf(e0, qa, sc[0]));
+        sc[1] = fmaf(sz1.x, d[1], fmaf(e1, qa, sc[1]));
+        sc[2] = fmaf(sz0.x, d[2], fmaf(e0, qb, sc[2]));
+        sc[3] = fmaf(sz1.x, d[3], fmaf(e1, qb, sc[3]));
+      }
+
+      // ---- masks, this warp's maximum, weights ----
+      float mloc[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int lim = (c < 2) ? lim0 : lim1;
+        const bool ok = page_ok && (P0 + tl0 + (c & 1)) < lim;
+        sc[c] = ok ? sc[c] * sl2 : -CUDART_INF_F;
+        mloc[c >> 1] = fmaxf(mloc[c >> 1], sc[c]);
+      }
+      float mw[2], l_own[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mloc[i] = fmaxf(mloc[i], __shfl_xor_sync(kFull, mloc[i], 1));
+        mloc[i] = fmaxf(mloc[i], __shfl_xor_sync(kFull, mloc[i], 2));
+        mw[i] = (mloc[i] > m_run[i] + kRescaleLog2) ? mloc[i] : m_run[i];
+      }
+      uint8_t* ptile = smem + Lo::kOffP + pb * kPTile;
+      {
+        const float meff0 = (mw[0] == -CUDART_INF_F) ? 0.0f : mw[0];
+        const float meff1 = (mw[1] == -CUDART_INF_F) ? 0.0f : mw[1];
+        const float2 p0 = make_float2(exp2f(sc[0] - meff0), exp2f(sc[1] - meff0));
+        const float2 p1 = make_float2(exp2f(sc[2] - meff1), exp2f(sc[3] - meff1));
+        l_own[0] = p0.x + p0.y;
+        l_own[1] = p1.x + p1.y;
+        *reinterpret_cast<float2*>(ptile + r * kPRow + tl0 * 4) = p0;
+        *reinterpret_cast<float2*>(ptile + (r + 8) * kPRow + tl0 * 4) = p1;
+      }
+      float* mt = reinterpret_cast<float*>(smem + Lo::kOffM) + pb * kRows * kWarps;
+      if (kp == 0) {
+        mt[r * kWarps + w] = mw[0];
+        mt[(r + 8) * kWarps + w] = mw[1];
+      }
+      named_barrier_compute();
+      if (tid == 0) issue_page(k + kNS - 1);
+
+      // ---- new running maximum; rescale O and the row sums when it moved ----
+      float mwr[2][kWarps];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float4 u = *reinterpret_cast<const float4*>(mt + (r + 8 * i) * kWarps);
+        const float4 v = *reinterpret_cast<const float4*>(mt + (r + 8 * i) * kWarps + 4);
+        mwr[i][0] = u.x; mwr[i][1] = u.y; mwr[i][2] = u.z; mwr[i][3] = u.w;
+        mwr[i][4] = v.x; mwr[i][5] = v.y; mwr[i][6] = v.z; mwr[i][7] = v.w;
+      }
+      float mnew[2], alpha[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        mnew[i] = m_run[i];
+#pragma unroll
+        for (int v = 0; v < kWarps; ++v) mnew[i] = fmaxf(mnew[i], mwr[i][v]);
+        alpha[i] = (mnew[i] == -CUDART_INF_F) ? 1.0f : exp2f(m_run[i] - mnew[i]);
+        const float own = (mw[i] == -CUDART_INF_F) ? 0.0f : exp2f(mw[i] - mnew[i]);
+        l_acc[i] = l_acc[i] * alpha[i] + l_own[i] * own;
+        corr[i] *= alpha[i];
+        m_run[i] = mnew[i];
+      }
+      if (__any_sync(kFull, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          o[j][0] *= alpha[0];
+          o[j][1] *= alpha[0];
+          o[j][2] *= alpha[1];
+          o[j][3] *= alpha[1];
+        }
+      }
+
+      // ---- O[16 rows, group w] += sum_t p_t c_hat_t over the page ----
+      // Block j, column n holds channel 64w + 8n + j: lane (r, kp) supplies
+      // column r from code word r of the group's 32 bytes. K-step ks takes keys
+      // 16ks + [0, 16), scored by warps 2ks and 2ks+1; their weights were taken
+      // against those warps' maxima and are scaled to the new one.
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const int ta = 16 * ks + 2 * kp, tb = ta + 8;  // page-local keys of B rows {0,1} and {8,9}
+        // weights in A-fragment order: (r, ta..ta+1), (r+8, ta..), (r, tb..), (r+8, tb..)
+        float2 pw[4] = {*reinterpret_cast<const float2*>(ptile + r * kPRow + ta * 4),
+                        *reinterpret_cast<const float2*>(ptile + (r + 8) * kPRow + ta * 4),
+                        *reinterpret_cast<const float2*>(ptile + r * kPRow + tb * 4),
+                        *reinterpret_cast<const float2*>(ptile + (r + 8) * kPRow + tb * 4)};
+        float fq[4];
+        bool scale_w = false;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float mq = mwr[q & 1][2 * ks + (q >> 1)];
+          fq[q] = (mq == -CUDART_INF_F) ? 0.0f : exp2f(mq - mnew[q & 1]);
+          scale_w |= fq[q] != 1.0f;
+        }
+        if (__any_sync(kFull, scale_w)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            pw[q].x *= fq[q];
+            pw[q].y *= fq[q];
+          }
+        }
+        // (s, z) of group w for keys ta, ta+1, tb, tb+1; keys past the end (or
+        // of a missing page) get s = z = 0, so garbage never reaches the MMA
+        float sv[4], zv[4];
+        uint32_t wd[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int t = (q < 2 ? ta : tb) + (q & 1);
+          const bool ok = page_ok && P0 + t < t_end;
+          const uint32_t m = ok ? *reinterpret_cast<const uint32_t*>(st + G::kOffCM + t * G::kGroupsC * 4 + 4 * w) : 0u;
+          const float2 sz = __half22float2(bits_h2(m));
+          sv[q] = sz.x;
+          zv[q] = sz.y;
+          wd[q] = *reinterpret_cast<const uint32_t*>(st + G::kOffCC + t * G::kRowC + 32 * w + 4 * r);
+        }
+        // A = w = p * s as fp16 hi + lo; the zero-point term sum p z in fp32
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k0 = (q < 2) ? 0 : 2;  // keys (ta, ta+1) or (tb, tb+1)
+          split_h2(pw[q].x * sv[k0], pw[q].y * sv[k0 + 1], ah[q], al[q]);
+          corr[q & 1] = fmaf(pw[q].x, zv[k0], fmaf(pw[q].y, zv[k0 + 1], corr[q & 1]));
+        }
+        // B: channel j of keys (ta, ta+1) and (tb, tb+1). The 16-bit pattern
+        // [u, 0x00] is the fp16 value u * 2^-24 (subnormal, exact): one byte
+        // permute per pair, no offset to cancel; the epilogue scales by 2^24.
+        const uint32_t la0 = wd[0] & 0x0F0F0F0Fu, ha0 = (wd[0] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t la1 = wd[1] & 0x0F0F0F0Fu, ha1 = (wd[1] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t lb0 = wd[2] & 0x0F0F0F0Fu, hb0 = (wd[2] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t lb1 = wd[3] & 0x0F0F0F0Fu, hb1 = (wd[3] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t sel = sel_pair(j >> 1);
+          const uint32_t b0 = (j & 1) ? prmt(ha0, ha1, sel) : prmt(la0, la1, sel);
+          const uint32_t b1 = (j & 1) ? prmt(hb0, hb1, sel) : prmt(lb0, lb1, sel);
+          mma_f16(o[j], ah, b0, b1);
+          mma_f16(o[j], al, b0, b1);
+        }
+      }
+    }
+
+    // ---- epilogue: row sums across lanes and warps, O / l, lse ----
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      l_acc[i] += __shfl_xor_sync(kFull, l_acc[i], 1);
+      l_acc[i] += __shfl_xor_sync(kFull, l_acc[i], 2);
+      corr[i] += __shfl_xor_sync(kFull, corr[i], 1);  // every lane of the row needs the group's full term
+      corr[i] += __shfl_xor_sync(kFull, corr[i], 2);
+    }
+    float* lt = reinterpret_cast<float*>(smem + Lo::kOffL);
+    if (kp == 0) {
+      lt[r * kWarps + w] = l_acc[0];
+      lt[(r + 8) * kWarps + w] = l_acc[1];
+    }
+    named_barrier_compute();  // also: every warp is done with the page stages
+    float l[2], inv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float4 u = *reinterpret_cast<const float4*>(lt + (r + 8 * i) * kWarps);
+      const float4 v = *reinterpret_cast<const float4*>(lt + (r + 8 * i) * kWarps + 4);
+      l[i] = ((u.x + u.y) + (u.z + u.w)) + ((v.x + v.y) + (v.z + v.w));
+      inv[i] = l[i] > 0.0f ? 1.0f / l[i] : 0.0f;
+    }
+    float* otile = reinterpret_cast<float*>(smem);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int ch = 64 * w + 8 * (2 * kp + e) + j;
+        otile[r * kORow + ch] = fmaf(o[j][e], kCodeScale, corr[0]) * inv[0];
+        otile[(r + 8) * kORow + ch] = fmaf(o[j][2 + e], kCodeScale, corr[1]) * inv[1];
+      }
+    }
+    const size_t part_row0 = (static_cast<size_t>(b) * a.n_split + split) * a.rows;
+    if (w == 0 && kp == 0) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int row = r + 8 * i;
+        if (row >= a.rows) continue;
+        const float lse = l[i] > 0.0f ? (m_run[i] + log2f(l[i])) * kLn2 : -CUDART_INF_F;
+        if (a.n_split == 1) {
+          if (a.lse) a.lse[static_cast<size_t>(b) * a.rows + row] = lse;
+        } else {
+          a.lse_part[part_row0 + row] = lse;
+        }
+      }
+    }
+    named_barrier_compute();
+    {
+      const int row = tid >> 4, seg = tid & 15;  // 16 rows x 16 segments of 32 channels
+      if (row < a.rows) {
+        const float* src = otile + row * kORow + seg * 32;
+        if (a.n_split == 1 && !a.out_f32) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                (static_cast<size_t>(b) * a.rows + row) * kDc + seg * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t wds[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(src[8 * v + 2 * e], src[8 * v + 2 * e + 1]);
+              wds[e] = *reinterpret_cast<uint32_t*>(&h);
+            }
+            dst[v] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+          }
+        } else {
+          float* base = (a.n_split == 1) ? static_cast<float*>(a.out) + (static_cast<size_t>(b) * a.rows + row) * kDc
+                                         : a.o_part + (part_row0 + row) * kDc;
+          float4* dst = reinterpret_cast<float4*>(base + seg * 32);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) dst[v] = make_float4(src[4 * v], src[4 * v + 1], src[4 * v + 2], src[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  // ---- teardown: after an abort, let every issued page copy land before the CTA exits ----
+  __syncthreads();
+  if (tid == 0 && *abort_flag) {
+    for (int k = max(0, n_issued - kNS); k < n_issued; ++k)
+      ptx::mbar_wait(&full[k % kNS], (k / kNS) & 1, nullptr, kWaitLimitNs);
+  }
+}
+
+template <int BC, int GC, int BR, int GR>
+cudaError_t launch_t(const DecodeLaunch& L) {
+  using Lo = Layout<QGeom<BC, GC, BR, GR>>;
+  auto kern = decode_small_kernel<BC, GC, BR, GR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lo::kBytes);
+  if (e != cudaSuccess) return e;
+  const DecodeArgs a = make_decode_args(L);
+  kern<<<static_cast<unsigned>(L.B * L.n_split), kThreads, Lo::kBytes, L.stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace small
+
+cudaError_t launch_decode_small(const DecodeLaunch& L) {
+  if (!L.quantized || L.s_q * L.H > small::kRows || L.num_pages < 1) return cudaErrorNotSupported;
+  if (L.bits_c == 4 && L.group_c == 64 && L.bits_r == 4 && L.group_r == 64) return small::launch_t<4, 64, 4, 64>(L);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace mla

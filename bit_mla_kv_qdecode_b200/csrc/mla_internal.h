@@ -56,5 +56,10 @@ cudaError_t launch_combine(const DecodeLaunch& L);
 // Returns cudaErrorNotSupported when the tensor-core kernel has no variant for
 // the shape; the caller then uses the SIMT kernel.
 cudaError_t launch_decode_tc(const DecodeLaunch& L);
+// Warp-level MMA kernel for s_q * H <= 16 rows (INT4 g64 content and RoPE);
+// cudaErrorNotSupported for other shapes and formats.
+cudaError_t launch_decode_small(const DecodeLaunch& L);
+// Query rows up to which a decode unit is one CTA of the small-row kernel.
+constexpr int kSmallRows = 16;
 
 }  // namespace mla

@@ -48,6 +48,11 @@ SMALL = [
     (4, 32, 2, 64, 32, 2, [100, 129]),
     (2, 64, 2, 32, 64, 1, [640, 64]),
     (4, 64, 4, 64, 8, 3, [3, 70]),
+    # at most 16 query rows: the warp-level MMA kernel (INT4 g64)
+    (4, 64, 4, 64, 16, 1, [1, 63, 64, 65, 200, 1000]),
+    (4, 64, 4, 64, 8, 2, [2, 65, 300, 4096]),
+    (4, 64, 4, 64, 5, 3, [100, 1, 129]),
+    (4, 64, 4, 64, 1, 1, [33, 640]),
 ]
 
 
