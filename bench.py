@@ -271,6 +271,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="dsv3")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run the workload with this many requests instead (small cases for profiling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
@@ -279,6 +281,8 @@ def main():
 
     from bit_mla_kv_qdecode_b200 import synth
     w = synth.workload(args.workload)
+    if args.batch > 0:
+        w = w.scaled(B=args.batch)
     if args.impl == "reference":
         return run_reference(args, w)
 
