@@ -120,6 +120,33 @@ def decode_bf16(pool_f32, table, seq_lens, qc, qr, scale: float, requests=None, 
     return o, lse
 
 
+def hybrid_decode(desc: layout.Desc, pool, table, hist_lens, prot_pool_f32, prot_table, prot_lens, qc, qr,
+                  scale: float, requests=None, page_size=64):
+    """Decode over a hybrid cache: BF16 protection of the earliest tokens and a
+    recent window, the history between them quantized; the history stays
+    visible, only its storage precision differs (QuantMLA podcast episode,
+    researchpod.app, the passage on keeping history uncompressed).
+    Per request b (readings, stated here): the protected segment holds
+    prot_lens[b] tokens of a BF16 pool in position order -- the sink, then the
+    window, the newest s_q keys last; the quantized pool holds the hist_lens[b]
+    history tokens, all older than every query. Query i sees every history key
+    and the first prot_lens[b] - s_q + 1 + i protected keys. One softmax over
+    both segments. qc, qr as in ``qdecode``; prot_pool_f32 [num_pages, P, d_c + d_r].
+    """
+    B, s_q, H = qc.shape[:3]
+    o = np.zeros((B, s_q, H, desc.d_c))
+    lse = np.full((B, s_q, H), -np.inf)
+    for b in (range(B) if requests is None else requests):
+        Th, Tp = int(hist_lens[b]), int(prot_lens[b])
+        Ch, Rh = layout.gather_tokens(desc, pool, table[b], Th)
+        Cp, Rp = layout.bf16_pool_gather(prot_pool_f32, prot_table[b], Tp, page_size, desc.d_c)
+        rq_c, rq_r, Lp = request_rows(qc[b], qr[b], Tp)
+        ob, lb = attend(rq_c, rq_r, np.concatenate([Ch, Cp]), np.concatenate([Rh, Rp]), scale, Th + Lp)
+        o[b] = ob.reshape(s_q, H, -1)
+        lse[b] = lb.reshape(s_q, H)
+    return o, lse
+
+
 def combine(o_parts, lse_parts):
     """Merge split-KV partial results.
 

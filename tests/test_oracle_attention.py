@@ -159,3 +159,75 @@ def test_paging_invariance_and_pool_decode():
         rq_c, rq_r, L = attention.request_rows(qc[b], qr[b], T)
         o, lse = attention.attend(rq_c, rq_r, Ch, Rh, SCALE, L)
         assert np.array_equal(outs[0][0][b].reshape(s_q * H, -1), o)
+
+
+def _bf16(x):
+    return (np.asarray(x, np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32)
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_hybrid_cache_equals_position_ordered_decode(s_q):
+    # The hybrid decode attends [history ; protected] with its own visibility
+    # rule. Restated independently: lay the tokens out by position -- sink
+    # (first k protected tokens), history, window (rest of the protected
+    # segment) -- each with its stored precision, and apply the ordinary causal
+    # rule L = T - s_q + 1 + i. Both must agree.
+    desc = layout.Desc()
+    rng = np.random.default_rng(21)
+    B, H, k = 2, 3, 64
+    hist = np.array([128, 0])
+    win = np.array([70, 5])
+    prot = k + win
+    T = hist + prot
+    c = _bf16(rng.standard_normal((B, T.max(), 512)))
+    r = _bf16(rng.standard_normal((B, T.max(), 64)))
+    qc, qr = _rand(rng, B, s_q, H, 512), _rand(rng, B, s_q, H, 64)
+    pool = layout.new_pool(desc, 4)
+    table = np.array([[0, 1], [2, 3]])
+    prot_pool = np.zeros((6, 64, 576), np.float32)
+    prot_table = np.array([[0, 1, 2], [3, 4, 5]])
+    for b in range(B):
+        hist_tok = slice(k, k + hist[b])
+        prot_tok = np.r_[0:k, k + hist[b]:T[b]]
+        if hist[b]:
+            layout.append(desc, pool, table[b:b + 1], [0], c[b:b + 1, hist_tok], r[b:b + 1, hist_tok])
+        rows = np.concatenate([c[b, prot_tok], r[b, prot_tok]], axis=1)
+        for j in range(prot[b]):
+            prot_pool[prot_table[b][j // 64], j % 64] = rows[j]
+    o, lse = attention.hybrid_decode(desc, pool, table, hist, prot_pool, prot_table, prot, qc, qr, SCALE)
+    for b in range(B):
+        C = c[b, :T[b]].astype(np.float64).copy()
+        R = r[b, :T[b]].astype(np.float64).copy()
+        if hist[b]:
+            from oracle import quant
+            u, s, z = quant.quantize_groups(c[b, k:k + hist[b]], 4, 64)
+            C[k:k + hist[b]] = quant.dequantize_groups(u, s, z, 64)
+            u, s, z = quant.quantize_groups(r[b, k:k + hist[b]], 4, 64)
+            R[k:k + hist[b]] = quant.dequantize_groups(u, s, z, 64)
+        rq_c, rq_r, L = attention.request_rows(qc[b], qr[b], T[b])
+        ob, lb = attention.attend(rq_c, rq_r, C, R, SCALE, L)
+        assert np.allclose(o[b].reshape(s_q * H, -1), ob, rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse[b].reshape(-1), lb, rtol=1e-12, atol=1e-12)
+
+
+def test_hybrid_cache_degenerate_segments():
+    # no history: the BF16 decode of the protected segment; no protected
+    # keys at s_q = 1: the quantized decode of the history
+    desc = layout.Desc()
+    rng = np.random.default_rng(22)
+    B, H, s_q = 1, 4, 1
+    c = _bf16(rng.standard_normal((B, 200, 512)))
+    r = _bf16(rng.standard_normal((B, 200, 64)))
+    qc, qr = _rand(rng, B, s_q, H, 512), _rand(rng, B, s_q, H, 64)
+    prot_pool = np.zeros((4, 64, 576), np.float32)
+    for j in range(200):
+        prot_pool[j // 64, j % 64] = np.concatenate([c[0, j], r[0, j]])
+    pt = np.array([[0, 1, 2, 3]])
+    pool = layout.new_pool(desc, 4)
+    layout.append(desc, pool, pt, [0], c, r)
+    o, lse = attention.hybrid_decode(desc, pool, pt, [0], prot_pool, pt, [200], qc, qr, SCALE)
+    o2, lse2 = attention.decode_bf16(prot_pool, pt, [200], qc, qr, SCALE)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    o, lse = attention.hybrid_decode(desc, pool, pt, [200], prot_pool, pt, [0], qc, qr, SCALE)
+    o3, lse3 = attention.qdecode(desc, pool, pt, [200], qc, qr, SCALE)
+    assert np.array_equal(o, o3) and np.array_equal(lse, lse3)

@@ -43,6 +43,9 @@ MUTANTS = [
     ("lse_without_log", "attention.py", "lse[live] = (m + np.log(l_))[:, 0]", "lse[live] = (m + l_)[:, 0]"),
     ("combine_weight_sign", "attention.py", "w = np.exp(lse_parts[:, live] - m[live][None, :])",
      "w = np.exp(m[live][None, :] - lse_parts[:, live])"),
+    ("hybrid_visibility", "attention.py", "scale, Th + Lp)", "scale, Th + Lp + 1)"),
+    ("hybrid_drops_history", "attention.py", "np.concatenate([Ch, Cp]), np.concatenate([Rh, Rp])",
+     "np.concatenate([Ch[:0], Cp]), np.concatenate([Rh[:0], Rp])"),
     ("query_rows_order", "attention.py", "return qc_b.reshape(s_q * H, -1), qr_b.reshape(s_q * H, -1), L",
      "return qc_b.transpose(1, 0, 2).reshape(s_q * H, -1), qr_b.reshape(s_q * H, -1), L"),
 ]
