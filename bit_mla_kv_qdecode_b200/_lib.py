@@ -57,6 +57,12 @@ SIGNATURES = {
                                  _c_void, _c_uint, _c_void]),
     "mla_qdecode_noalloc": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void, _c_int,
                                      _c_int, _c_int, _c_float, _c_int, _c_void, _c_int, _c_void, _c_uint, _c_void]),
+    "mla_qcache_append_bf16_pages": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_void, _c_int, _c_void,
+                                              _c_int, _c_void]),
+    "mla_qdecode_hybrid_workspace_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "mla_qdecode_hybrid": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_int, _c_void,
+                                    _c_int, _c_void, _c_int, _c_void, _c_void, _c_int, _c_int, _c_int, _c_float,
+                                    _c_void, _c_size, _c_void, _c_int, _c_void, _c_void]),
     "mla_get_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_void]),
 }
 

@@ -147,6 +147,46 @@ def mla_decode_bf16(pool, block_table, seq_lens, max_seq_len, q_c, q_r, scale, *
     return out, lse
 
 
+def mla_qcache_append_bf16_pages(desc, pool, block_table, seq_lens_before, bf16_pool, src_pages, stream=None) -> None:
+    """Quantize whole BF16 pages (src_pages[b] of bf16_pool, or -1) into the quantized cache at
+    positions seq_lens_before[b] .. + 63. See include/mla_qcache.h."""
+    B = src_pages.shape[0]
+    check("mla_qcache_append_bf16_pages", _lib.load().mla_qcache_append_bf16_pages(
+        ctypes.byref(desc), _need(pool, "pool", torch.uint8), _need(block_table, "block_table", torch.int32),
+        block_table.shape[1], _need(seq_lens_before, "seq_lens_before", torch.int32, (B,)),
+        _need(bf16_pool, "bf16_pool", torch.bfloat16), bf16_pool.shape[0],
+        _need(src_pages, "src_pages", torch.int32, (B,)), B, _stream(stream)))
+
+
+def mla_qdecode_hybrid_workspace_bytes(B, s_q, H, max_hist_len, max_prot_len) -> int:
+    return int(_lib.load().mla_qdecode_hybrid_workspace_bytes(B, s_q, H, max_hist_len, max_prot_len))
+
+
+def mla_qdecode_hybrid(desc, pool, block_table, hist_lens, max_hist_len, bf16_pool, prot_table, prot_lens,
+                       max_prot_len, q_c, q_r, scale, *, out=None, out_dtype=torch.bfloat16, lse=None,
+                       workspace=None, stream=None):
+    """Decode over a hybrid cache (quantized history + BF16 sink and window). Returns (out, lse)."""
+    B, s_q, H = q_c.shape[:3]
+    qc = _need(q_c, "q_c", torch.bfloat16, (B, s_q, H, D_C))
+    qr = _need(q_r, "q_r", torch.bfloat16, (B, s_q, H, D_R))
+    if out is None:
+        out = torch.empty((B, s_q, H, D_C), dtype=out_dtype, device=q_c.device)
+    po = _need(out, "out", out.dtype, (B, s_q, H, D_C))
+    pl = None if lse is None else _need(lse, "lse", torch.float32, (B, s_q, H))
+    need = mla_qdecode_hybrid_workspace_bytes(B, s_q, H, max_hist_len, max_prot_len)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q_c.device)
+    check("mla_qdecode_hybrid", _lib.load().mla_qdecode_hybrid(
+        ctypes.byref(desc), _need(pool, "pool", torch.uint8), _need(block_table, "block_table", torch.int32),
+        block_table.shape[1], _need(hist_lens, "hist_lens", torch.int32, (B,)), int(max_hist_len),
+        _need(bf16_pool, "bf16_pool", torch.bfloat16), bf16_pool.shape[0],
+        _need(prot_table, "prot_table", torch.int32), prot_table.shape[1],
+        _need(prot_lens, "prot_lens", torch.int32, (B,)), int(max_prot_len), qc, qr, B, s_q, H, float(scale),
+        _need(workspace, "workspace", torch.uint8), workspace.numel(), po, int(out.dtype == torch.float32), pl,
+        _stream(stream)))
+    return out, lse
+
+
 def mla_get_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     check("mla_get_device_status", _lib.load().mla_get_device_status(ctypes.byref(v), _stream(stream)))

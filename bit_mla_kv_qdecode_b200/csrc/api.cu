@@ -96,6 +96,26 @@ size_t workspace_for(int B, int rows, const SplitPlan& p) {
 
 mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
 
+// Hybrid decode workspace: the two segments' fp32 results and lse, then the
+// scratch their decodes share (they run one after the other on one stream).
+struct HybridWorkspace {
+  size_t off_o_hist, off_l_hist, off_o_prot, off_l_prot, off_inner, inner, total;
+};
+
+HybridWorkspace hybrid_workspace(int B, int s_q, int H, int max_hist_len, int max_prot_len) {
+  const size_t rows = static_cast<size_t>(B) * s_q * H;
+  HybridWorkspace w{};
+  w.off_o_hist = 0;
+  w.off_l_hist = align_up(w.off_o_hist + rows * mla::kDc * sizeof(float), 256);
+  w.off_o_prot = align_up(w.off_l_hist + rows * sizeof(float), 256);
+  w.off_l_prot = align_up(w.off_o_prot + rows * mla::kDc * sizeof(float), 256);
+  w.off_inner = align_up(w.off_l_prot + rows * sizeof(float), 256);
+  w.inner = std::max(workspace_for(B, s_q * H, plan_splits(B, 1, s_q * H, max_hist_len, 0)),
+                     workspace_for(B, s_q * H, plan_splits(B, s_q, H, max_prot_len, 0)));
+  w.total = w.off_inner + w.inner;
+  return w;
+}
+
 struct DecodeCommon {
   const void* pool;
   int num_pages;
@@ -258,8 +278,28 @@ mla_status mla_qcache_append(const mla_qcache_desc* desc, void* pool, const int3
   int* status = status_ptr();
   if (!status) return MLA_ERR_CUDA;
   mla::AppendLaunch L{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens_before, c_new, kr_new,
-                      B, n_new, desc->bits_c, desc->group_c, desc->bits_r, desc->group_r, status,
-                      reinterpret_cast<cudaStream_t>(stream)};
+                      B, n_new, desc->bits_c, desc->group_c, desc->bits_r, desc->group_r,
+                      nullptr, 0, nullptr, status, reinterpret_cast<cudaStream_t>(stream)};
+  return from_cuda(mla::launch_qcache_append(L));
+}
+
+mla_status mla_qcache_append_bf16_pages(const mla_qcache_desc* desc, void* pool, const int32_t* block_table,
+                                        int max_pages_per_seq, const int32_t* seq_lens_before,
+                                        const void* bf16_pool, int bf16_num_pages, const int32_t* src_pages, int B,
+                                        mla_stream_t stream) {
+  const mla_status st = mla_qcache_check_desc(desc);
+  if (st != MLA_OK) return st;
+  if (B < 0 || bf16_num_pages < 0) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!pool || !block_table || !seq_lens_before || !src_pages || max_pages_per_seq < 1) return MLA_ERR_INVALID_ARG;
+  if (bf16_num_pages > 0 && !bf16_pool) return MLA_ERR_INVALID_ARG;
+  if (!aligned(pool, 256) || !aligned(bf16_pool, 16)) return MLA_ERR_INVALID_ARG;
+  if (B > (1 << 20)) return MLA_ERR_UNSUPPORTED;
+  int* status = status_ptr();
+  if (!status) return MLA_ERR_CUDA;
+  mla::AppendLaunch L{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens_before, nullptr, nullptr,
+                      B, mla::kPage, desc->bits_c, desc->group_c, desc->bits_r, desc->group_r,
+                      bf16_pool, bf16_num_pages, src_pages, status, reinterpret_cast<cudaStream_t>(stream)};
   return from_cuda(mla::launch_qcache_append(L));
 }
 
@@ -276,7 +316,7 @@ mla_status mla_bf16cache_append(void* pool, int num_pages, int page_size, const 
   int* status = status_ptr();
   if (!status) return MLA_ERR_CUDA;
   mla::AppendLaunch L{pool, num_pages, block_table, max_pages_per_seq, seq_lens_before, c_new, kr_new,
-                      B, n_new, 0, 0, 0, 0, status, reinterpret_cast<cudaStream_t>(stream)};
+                      B, n_new, 0, 0, 0, 0, nullptr, 0, nullptr, status, reinterpret_cast<cudaStream_t>(stream)};
   return from_cuda(mla::launch_bf16cache_append(L));
 }
 
@@ -313,6 +353,46 @@ mla_status mla_decode_bf16(const void* pool, int num_pages, int page_size, const
                  B, s_q, H, scale, num_splits, workspace, workspace_bytes, out, out_dtype, lse, flags,
                  reinterpret_cast<cudaStream_t>(stream)};
   return run_decode(c, false, nullptr);
+}
+
+size_t mla_qdecode_hybrid_workspace_bytes(int B, int s_q, int H, int max_hist_len, int max_prot_len) {
+  if (B <= 0 || s_q < 1 || H < 1 || max_hist_len < 0 || max_prot_len < 0) return 0;
+  return hybrid_workspace(B, s_q, H, max_hist_len, max_prot_len).total;
+}
+
+mla_status mla_qdecode_hybrid(const mla_qcache_desc* desc, const void* pool, const int32_t* block_table,
+                              int max_pages_per_seq, const int32_t* hist_lens, int max_hist_len,
+                              const void* bf16_pool, int bf16_num_pages, const int32_t* prot_table,
+                              int prot_max_pages, const int32_t* prot_lens, int max_prot_len, const void* q_c,
+                              const void* q_r, int B, int s_q, int H, float scale, void* workspace,
+                              size_t workspace_bytes, void* out, int out_dtype, float* lse, mla_stream_t stream) {
+  const mla_status st = mla_qcache_check_desc(desc);
+  if (st != MLA_OK) return st;
+  if (B < 0 || s_q < 1 || H < 1 || max_hist_len < 0 || max_prot_len < 0) return MLA_ERR_INVALID_ARG;
+  if (out_dtype != 0 && out_dtype != 1) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (!out || !q_c || !q_r || !aligned(out, 16) || !aligned(lse, 4)) return MLA_ERR_INVALID_ARG;
+  const HybridWorkspace hw = hybrid_workspace(B, s_q, H, max_hist_len, max_prot_len);
+  if (!workspace || workspace_bytes < hw.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+  char* base = static_cast<char*>(workspace);
+  float* o_hist = reinterpret_cast<float*>(base + hw.off_o_hist);
+  float* l_hist = reinterpret_cast<float*>(base + hw.off_l_hist);
+  float* o_prot = reinterpret_cast<float*>(base + hw.off_o_prot);
+  float* l_prot = reinterpret_cast<float*>(base + hw.off_l_prot);
+  void* inner = hw.inner ? base + hw.off_inner : nullptr;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // history: every key is older than every query, so its rows are decoded as
+  // s_q * H rows of one query position (no causal offset)
+  DecodeCommon ch{pool, desc->num_pages, block_table, max_pages_per_seq, hist_lens, max_hist_len, q_c, q_r,
+                  B, 1, s_q * H, scale, 0, inner, hw.inner, o_hist, 1, l_hist, 0, s};
+  mla_status r = run_decode(ch, true, desc);
+  if (r != MLA_OK) return r;
+  // protected segment: position order, the newest s_q keys last (causal)
+  DecodeCommon cp{bf16_pool, bf16_num_pages, prot_table, prot_max_pages, prot_lens, max_prot_len, q_c, q_r,
+                  B, s_q, H, scale, 0, inner, hw.inner, o_prot, 1, l_prot, 0, s};
+  r = run_decode(cp, false, nullptr);
+  if (r != MLA_OK) return r;
+  return from_cuda(mla::launch_merge2(o_hist, l_hist, o_prot, l_prot, B * s_q * H, out, out_dtype, lse, s));
 }
 
 mla_status mla_get_device_status(int* status, mla_stream_t stream) {

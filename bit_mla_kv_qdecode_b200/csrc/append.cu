@@ -36,12 +36,29 @@ __global__ void __launch_bounds__(256)
 qcache_append_kernel(uint8_t* __restrict__ pool, int num_pages, const int32_t* __restrict__ table,
                      int max_pages, const int32_t* __restrict__ lens_before,
                      const __nv_bfloat16* __restrict__ c_new, const __nv_bfloat16* __restrict__ kr_new,
-                     int n_tokens, int n_new, int* status) {
+                     const __nv_bfloat16* __restrict__ src_pool, int src_num_pages,
+                     const int32_t* __restrict__ src_pages, int n_tokens, int n_new, int* status) {
   using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
   const int lane = threadIdx.x & 31;
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (tok >= n_tokens) return;
   const int b = tok / n_new, j = tok - b * n_new;
+  // token source: the dense arrays, or row j of BF16 page src_pages[b] ([64][576], content then RoPE)
+  const __nv_bfloat16* c_src;
+  const __nv_bfloat16* kr_src;
+  if (!src_pages) {
+    c_src = c_new + static_cast<size_t>(tok) * kDc;
+    kr_src = kr_new + static_cast<size_t>(tok) * kDr;
+  } else {
+    const int sp = __ldg(src_pages + b);
+    if (sp < 0) return;  // this request moves nothing
+    if (sp >= src_num_pages) {
+      if (lane == 0) record_error(status, MLA_ERR_INVALID_ARG);
+      return;
+    }
+    c_src = src_pool + (static_cast<size_t>(sp) * kPage + j) * kDqk;
+    kr_src = c_src + kDc;
+  }
   const int t = __ldg(lens_before + b) + j;
   const int page = lookup_page(table, max_pages, num_pages, b, t);
   if (page < 0) {
@@ -52,7 +69,7 @@ qcache_append_kernel(uint8_t* __restrict__ pool, int num_pages, const int32_t* _
   uint8_t* pg = pool + static_cast<size_t>(page) * G::kPageBytes;
 
   // ---- content path: 16 channels per lane ----
-  const uint4* src = reinterpret_cast<const uint4*>(c_new + static_cast<size_t>(tok) * kDc) + 2 * lane;
+  const uint4* src = reinterpret_cast<const uint4*>(c_src) + 2 * lane;
   const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
   const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
   float x[16];
@@ -96,7 +113,7 @@ qcache_append_kernel(uint8_t* __restrict__ pool, int num_pages, const int32_t* _
   }
 
   // ---- RoPE path: 2 channels per lane ----
-  const uint32_t rw = __ldg(reinterpret_cast<const uint32_t*>(kr_new + static_cast<size_t>(tok) * kDr) + lane);
+  const uint32_t rw = __ldg(reinterpret_cast<const uint32_t*>(kr_src) + lane);
   const float r0 = bf16_lo(rw), r1 = bf16_hi(rw);
   float rmn = fminf(r0, r1), rmx = fmaxf(r0, r1);
   constexpr int kLanesR = G_R / 2;
@@ -154,7 +171,7 @@ static cudaError_t launch_append_t(const AppendLaunch& L) {
   qcache_append_kernel<BC, GC, BR, GR><<<blocks, 256, 0, L.stream>>>(
       static_cast<uint8_t*>(L.pool), L.num_pages, L.table, L.max_pages, L.lens_before,
       static_cast<const __nv_bfloat16*>(L.c_new), static_cast<const __nv_bfloat16*>(L.kr_new),
-      n_tokens, L.n_new, L.status);
+      static_cast<const __nv_bfloat16*>(L.src_pool), L.src_num_pages, L.src_pages, n_tokens, L.n_new, L.status);
   return cudaGetLastError();
 }
 

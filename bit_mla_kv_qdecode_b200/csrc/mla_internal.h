@@ -16,6 +16,11 @@ struct AppendLaunch {
   const void* kr_new;
   int B, n_new;
   int bits_c, group_c, bits_r, group_r;
+  // optional token source for the quantized append: row j of BF16 page
+  // src_pages[b] of src_pool ([pages][64][576]) instead of c_new / kr_new
+  const void* src_pool;
+  int src_num_pages;
+  const int32_t* src_pages;
   int* status;
   cudaStream_t stream;
 };
@@ -52,6 +57,10 @@ struct DecodeArgs;
 DecodeArgs make_decode_args(const DecodeLaunch& L);
 
 cudaError_t launch_decode_simt(const DecodeLaunch& L);
+// out = log-sum-exp merge of two normalised partial results (fp32 [rows][512]
+// each, natural-log lse; -inf carries weight 0), as bf16 (out_f32 = 0) or fp32.
+cudaError_t launch_merge2(const float* o_a, const float* l_a, const float* o_b, const float* l_b, int rows,
+                          void* out, int out_f32, float* lse, cudaStream_t stream);
 cudaError_t launch_combine(const DecodeLaunch& L);
 // Returns cudaErrorNotSupported when the tensor-core kernel has no variant for
 // the shape; the caller then uses the SIMT kernel.

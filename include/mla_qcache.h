@@ -242,6 +242,71 @@ mla_status mla_qdecode_noalloc(const mla_qcache_desc* desc, const void* pool,
                                void* out, int out_dtype, float* lse,
                                unsigned flags, mla_stream_t stream);
 
+/* ---- Hybrid cache: BF16 protection of the earliest tokens and a recent window ----
+ *
+ * QuantMLA keeps the earliest tokens and a recent window in BF16 and the
+ * history between them in the low-bit cache; history stays visible, only its
+ * storage precision differs (QuantMLA podcast episode, the passage on keeping
+ * history uncompressed). The pages fix neither sizes nor layout. This library
+ * reads them as two caches per request:
+ *   protected segment  a BF16 cache (pool and block table as for
+ *                      mla_bf16cache_append / mla_decode_bf16) holding the
+ *                      sink and the window in position order, newest last;
+ *   history            the quantized cache (as for mla_qdecode) holding the
+ *                      tokens between them, all older than every query.
+ * Tokens enter the window with mla_bf16cache_append and leave it a whole page
+ * at a time with mla_qcache_append_bf16_pages; the caller owns both block
+ * tables and the page bookkeeping. */
+
+/* Quantize whole BF16 pages into the quantized cache: for each request b with
+ * src_pages[b] >= 0, the 64 tokens of page src_pages[b] of bf16_pool are
+ * quantized and packed exactly as mla_qcache_append would pack them, and
+ * written at positions seq_lens_before[b] .. seq_lens_before[b] + 63 of request
+ * b's quantized cache. Requests with src_pages[b] < 0 are skipped.
+ *   desc, pool, block_table, max_pages_per_seq, seq_lens_before
+ *                     as for mla_qcache_append (device pointers).
+ *   bf16_pool         device bf16 [bf16_num_pages, 64, 576], 16-byte aligned.
+ *   src_pages         device int32 [B]; entries >= bf16_num_pages are skipped
+ *                     and flagged in the device status word.
+ * Reads the BF16 pages, writes only the quantized pool. B == 0 is a no-op. */
+mla_status mla_qcache_append_bf16_pages(const mla_qcache_desc* desc, void* pool,
+                                        const int32_t* block_table, int max_pages_per_seq,
+                                        const int32_t* seq_lens_before,
+                                        const void* bf16_pool, int bf16_num_pages,
+                                        const int32_t* src_pages, int B, mla_stream_t stream);
+
+/* Workspace bytes mla_qdecode_hybrid needs (0 for invalid arguments). */
+size_t mla_qdecode_hybrid_workspace_bytes(int B, int s_q, int H, int max_hist_len,
+                                          int max_prot_len);
+
+/* Decode over a hybrid cache: one softmax over request b's hist_lens[b]
+ * quantized history keys and prot_lens[b] BF16 protected keys. Query i sees
+ * every history key and the first prot_lens[b] - s_q + 1 + i protected keys
+ * (the protected segment ends with the s_q newest keys, so the window must
+ * hold at least s_q tokens). Output and lse as for mla_qdecode.
+ *   desc, pool, block_table, max_pages_per_seq
+ *                     the quantized history cache (as for mla_qdecode);
+ *   hist_lens         device int32 [B], in [0, max_hist_len];
+ *   bf16_pool, bf16_num_pages, prot_table, prot_max_pages
+ *                     the protected segment's BF16 cache (page size 64);
+ *   prot_lens         device int32 [B], in [0, max_prot_len];
+ *   q_c, q_r, B, s_q, H, scale, out, out_dtype, lse  as for mla_qdecode;
+ *   workspace         device, 256-byte aligned, at least
+ *                     mla_qdecode_hybrid_workspace_bytes(...) bytes.
+ * The two segments are decoded one after the other (auto split plans) into
+ * fp32 partial results in the workspace and merged by log-sum-exp.
+ * Errors as for mla_qdecode; MLA_ERR_WORKSPACE if the workspace is short. */
+mla_status mla_qdecode_hybrid(const mla_qcache_desc* desc, const void* pool,
+                              const int32_t* block_table, int max_pages_per_seq,
+                              const int32_t* hist_lens, int max_hist_len,
+                              const void* bf16_pool, int bf16_num_pages,
+                              const int32_t* prot_table, int prot_max_pages,
+                              const int32_t* prot_lens, int max_prot_len,
+                              const void* q_c, const void* q_r,
+                              int B, int s_q, int H, float scale,
+                              void* workspace, size_t workspace_bytes,
+                              void* out, int out_dtype, float* lse, mla_stream_t stream);
+
 /* Read and clear the current device's status word: waits for `stream`, then
  * stores into *status the first error any kernel recorded since the last
  * read (MLA_OK if none). status is host memory. */
