@@ -65,6 +65,10 @@ def profiled_traffic(workload_name):
     return rec["dram_bytes_read_per_launch"] + rec["dram_bytes_write_per_launch"]
 
 
+HYB_SINK = 64      # BF16 sink of the hybrid cache leg: one page
+HYB_WINDOW = 128   # BF16 recent window: 128..191 tokens (history moves a page at a time)
+
+
 def max_over_ranks(x, dist, device):
     """The largest of every rank's x: a multi-rank job ends when its slowest rank does."""
     import torch
@@ -276,6 +280,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
+    ap.add_argument("--no-hybrid", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -323,8 +328,14 @@ def main():
     pool_b0 = api.new_bf16_pool(num_pages, device=dev) if want_bf16 else None
     new_c = np.zeros((w.B, w.n_new, 512), dtype=np.uint16)
     new_r = np.zeros((w.B, w.n_new, 64), dtype=np.uint16)
+    # hybrid cache leg: a one-page BF16 sink, a BF16 window of HYB_WINDOW..+63
+    # tokens, the history between them quantized (a page at a time)
+    hyb_hist = np.maximum((lens.astype(np.int64) - HYB_SINK - HYB_WINDOW) // 64 * 64, 0)
+    hyb_prot = []
     for b in range(w.B):
         toks = synth.cache_tokens_bf16(w, b, int(lens[b]), mag)
+        if not args.no_hybrid:
+            hyb_prot.append(np.concatenate([toks[:HYB_SINK], toks[HYB_SINK + hyb_hist[b]:]]))
         for t0 in range(0, int(lens[b]), 16384):
             part = toks[t0:t0 + 16384]
             lb = torch.tensor([t0], dtype=torch.int32, device=dev)
@@ -425,6 +436,46 @@ def main():
                     "qdecode_speedup": ms_b / ms_decode}
         del pools_b
 
+    # ---- hybrid cache decode (same queries and keys; history = the pool's pages after the sink page) ----
+    hybrid_leg = None
+    if not args.no_hybrid:
+        prot_lens = np.array([len(p) for p in hyb_prot], dtype=np.int32)
+        pp = int((prot_lens.max() + 63) // 64)
+        bpool_h = api.new_bf16_pool(w.B * pp, device=dev)
+        ptab = torch.arange(w.B * pp, dtype=torch.int32, device=dev).view(w.B, pp)
+        for b in range(w.B):
+            pt = to_dev(hyb_prot[b][None])
+            api.mla_bf16cache_append(bpool_h, ptab[b:b + 1], torch.zeros(1, dtype=torch.int32, device=dev),
+                                     pt[..., :512].contiguous(), pt[..., 512:].contiguous())
+        htab = table_t[:, HYB_SINK // 64:].contiguous()
+        hl_t = torch.from_numpy(hyb_hist.astype(np.int32)).to(dev)
+        pl_t = torch.from_numpy(prot_lens).to(dev)
+        mh, mp = int(hyb_hist.max()), int(prot_lens.max())
+        ws_h = torch.empty(max(api.mla_qdecode_hybrid_workspace_bytes(w.B, w.s_q, w.H, mh, mp), 1),
+                           dtype=torch.uint8, device=dev)
+
+        def hyb(k):
+            api.mla_qdecode_hybrid(desc, pools[k], htab, hl_t, mh, bpool_h, ptab, pl_t, mp, qcs[k], qrs[k], w.scale,
+                                   out=out, lse=lse, workspace=ws_h, stream=stream)
+
+        for i in range(args.warmup):
+            hyb(i % R)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            hyb(i % R)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert api.mla_get_device_status() == 0
+        ms_h = e0.elapsed_time(e1) / args.steps
+        q_bytes = int(hyb_hist.sum()) * page_bytes // 64
+        b_bytes = int(prot_lens.sum()) * 1152
+        hybrid_leg = {"sink": HYB_SINK, "window": f"{HYB_WINDOW}..{HYB_WINDOW + 63}", "ms_per_decode": ms_h,
+                      "head_tokens_per_s": st["head_tokens"] / (ms_h * 1e-3), "vs_qdecode_time": ms_h / ms_decode,
+                      "cache_bytes": q_bytes + b_bytes,
+                      "compression_vs_bf16": int(lens.astype(np.int64).sum()) * 1152 / (q_bytes + b_bytes)}
+
     # ---- end to end through the C ABI with host buffers ----
     h_qc = torch.from_numpy(qc_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     h_qr = torch.from_numpy(qr_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -477,6 +528,7 @@ def main():
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches_per_step * args.steps,
         "bf16_decode": bf16_leg,
+        "hybrid_decode": hybrid_leg,
         "clocks": clk.summary(),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
