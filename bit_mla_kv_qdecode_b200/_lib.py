@@ -63,6 +63,8 @@ SIGNATURES = {
     "mla_qdecode_hybrid": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_int, _c_void,
                                     _c_int, _c_void, _c_int, _c_void, _c_void, _c_int, _c_int, _c_int, _c_float,
                                     _c_void, _c_size, _c_void, _c_int, _c_void, _c_void]),
+    "mla_cache_bytes_per_request": (_c_size, [_P, ctypes.c_long, _c_int, _c_int]),
+    "mla_cache_max_requests": (ctypes.c_long, [_P, ctypes.c_long, _c_int, _c_int, _c_size]),
     "mla_get_device_status": (_c_int, [ctypes.POINTER(_c_int), _c_void]),
 }
 

@@ -187,6 +187,17 @@ def mla_qdecode_hybrid(desc, pool, block_table, hist_lens, max_hist_len, bf16_po
     return out, lse
 
 
+def mla_cache_bytes_per_request(desc, seq_len, sink=0, window=0) -> int:
+    """Bytes one request holds (desc None: the BF16 cache). See include/mla_qcache.h."""
+    return int(_lib.load().mla_cache_bytes_per_request(None if desc is None else ctypes.byref(desc),
+                                                       int(seq_len), int(sink), int(window)))
+
+
+def mla_cache_max_requests(desc, seq_len, budget_bytes, sink=0, window=0) -> int:
+    return int(_lib.load().mla_cache_max_requests(None if desc is None else ctypes.byref(desc), int(seq_len),
+                                                  int(sink), int(window), int(budget_bytes)))
+
+
 def mla_get_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     check("mla_get_device_status", _lib.load().mla_get_device_status(ctypes.byref(v), _stream(stream)))

@@ -395,6 +395,32 @@ mla_status mla_qdecode_hybrid(const mla_qcache_desc* desc, const void* pool, con
   return from_cuda(mla::launch_merge2(o_hist, l_hist, o_prot, l_prot, B * s_q * H, out, out_dtype, lse, s));
 }
 
+size_t mla_cache_bytes_per_request(const mla_qcache_desc* desc, long seq_len, int sink, int window) {
+  constexpr size_t kBf16Page = static_cast<size_t>(mla::kPage) * mla::kDqk * 2;
+  if (seq_len < 0 || sink < 0 || window < 0 || sink % mla::kPage != 0) return 0;
+  auto pages = [](long n) { return static_cast<size_t>((n + mla::kPage - 1) / mla::kPage); };
+  if (!desc) {
+    if (sink || window) return 0;
+    return pages(seq_len) * kBf16Page;
+  }
+  mla_qcache_desc d = *desc;
+  d.num_pages = 0;
+  const size_t qpage = mla_qcache_page_bytes(&d);
+  if (qpage == 0) return 0;
+  if (sink == 0 && window == 0) return pages(seq_len) * qpage;
+  const long hist = std::max(0L, (seq_len - sink - window) / mla::kPage * mla::kPage);
+  const long prot_sink = std::min<long>(sink, seq_len);
+  const long prot_window = seq_len - prot_sink - hist;
+  return pages(hist) * qpage + (pages(prot_sink) + pages(prot_window)) * kBf16Page;
+}
+
+long mla_cache_max_requests(const mla_qcache_desc* desc, long seq_len, int sink, int window,
+                            size_t budget_bytes) {
+  const size_t per = mla_cache_bytes_per_request(desc, seq_len, sink, window);
+  if (per == 0) return -1;  // invalid arguments, or an empty request (no bound)
+  return static_cast<long>(budget_bytes / per);
+}
+
 mla_status mla_get_device_status(int* status, mla_stream_t stream) {
   if (!status) return MLA_ERR_INVALID_ARG;
   *status = MLA_OK;

@@ -307,6 +307,25 @@ mla_status mla_qdecode_hybrid(const mla_qcache_desc* desc, const void* pool,
                               void* workspace, size_t workspace_bytes,
                               void* out, int out_dtype, float* lse, mla_stream_t stream);
 
+/* ---- Cache capacity (host arithmetic, no device work) ----
+ *
+ * Bytes one request of seq_len tokens holds in whole pages: the quantized
+ * layout of desc (its num_pages is ignored), or the BF16 cache if desc is NULL
+ * (1152 bytes per token). With sink > 0 or window > 0 (desc only), the hybrid
+ * policy of mla_qdecode_hybrid as read here: the first `sink` tokens (a whole
+ * number of pages) and the newest window .. window + 63 tokens in BF16 pages,
+ * the history between them -- 64 * floor((seq_len - sink - window) / 64)
+ * tokens -- in quantized pages. Returns 0 for invalid arguments (negative
+ * sizes, sink not a multiple of the page size, an unsupported desc). */
+size_t mla_cache_bytes_per_request(const mla_qcache_desc* desc, long seq_len, int sink, int window);
+
+/* Largest number of requests of seq_len tokens whose caches fit together in
+ * budget_bytes (no page sharing between requests), or -1 for invalid
+ * arguments or seq_len == 0 (no bound). The capacity side of the pages' cache-pressure serving result:
+ * a format that admits more concurrent requests avoids preemption. */
+long mla_cache_max_requests(const mla_qcache_desc* desc, long seq_len, int sink, int window,
+                            size_t budget_bytes);
+
 /* Read and clear the current device's status word: waits for `stream`, then
  * stores into *status the first error any kernel recorded since the last
  * read (MLA_OK if none). status is host memory. */

@@ -119,3 +119,33 @@ def test_decode_argument_errors(lib):
     assert lib.mla_decode_bf16(FAKE, 8, 64, FAKE, 4, FAKE, 300, FAKE, FAKE, 2, 1, 16, 0.1, 1, None, 0, FAKE, 0,
                                None, 0, None) == E.MLA_ERR_CAPACITY
     assert lib.mla_get_device_status(None, None) == E.MLA_ERR_INVALID_ARG
+
+
+def test_cache_capacity_closed_forms(lib):
+    # host arithmetic only: bytes per request in whole pages, and requests per budget
+    from bit_mla_kv_qdecode_b200 import api
+    T = 131072
+    d44 = api.make_desc(4, 64, 4, 64, num_pages=7)  # num_pages is ignored
+    d24 = api.make_desc(2, 32, 4, 64)
+    assert api.mla_cache_bytes_per_request(None, T) == T * 1152
+    assert api.mla_cache_bytes_per_request(d44, T) == T * 324  # 2048 pages x 20,736 B
+    assert api.mla_cache_bytes_per_request(d24, T) == T * 228
+    assert api.mla_cache_bytes_per_request(d44, 65) == 2 * 20736  # whole pages
+    # hybrid: sink 64 + window 128..191 in BF16 pages, history 64 * floor((T - 192) / 64) quantized
+    hist = (T - 192) // 64 * 64
+    assert hist == T - 192
+    assert api.mla_cache_bytes_per_request(d44, T, 64, 128) == (hist // 64) * 20736 + (1 + 2) * 64 * 1152
+    assert api.mla_cache_bytes_per_request(d44, 100, 64, 128) == 2 * 64 * 1152  # all protected
+    assert api.mla_cache_bytes_per_request(d44, 1000, 64, 128) == 12 * 20736 + (1 + 3) * 64 * 1152
+    ratio = api.mla_cache_bytes_per_request(None, T) / api.mla_cache_bytes_per_request(d44, T, 64, 128)
+    assert 3.54 < ratio < 3.556
+    # requests per budget: floor(budget / bytes)
+    budget = 140 * 10 ** 9
+    assert api.mla_cache_max_requests(None, T, budget) == budget // (T * 1152)
+    assert api.mla_cache_max_requests(d44, T, budget) == budget // (T * 324)
+    assert api.mla_cache_max_requests(d24, T, budget) == budget // (T * 228)
+    # invalid: sink not a whole number of pages, negative sizes, protection without a desc, empty request
+    assert api.mla_cache_bytes_per_request(d44, T, 10, 0) == 0
+    assert api.mla_cache_bytes_per_request(d44, -1) == 0
+    assert api.mla_cache_bytes_per_request(None, T, 64, 0) == 0
+    assert api.mla_cache_max_requests(d44, 0, budget) == -1
