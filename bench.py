@@ -481,37 +481,64 @@ def main():
     h_qr = torch.from_numpy(qr_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     h_nc = torch.from_numpy(new_c.view(np.int16)).view(torch.bfloat16).pin_memory()
     h_nr = torch.from_numpy(new_r.view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    d_nc, d_nr = torch.empty_like(newc_t), torch.empty_like(newr_t)
+    # Double-buffered: step k's uploads (on their own stream) overlap step k-1's
+    # append + decode, and its read-back (another stream) overlaps step k+1's.
+    # Every step still moves its inputs in and its output and lse out.
+    hs, ds = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    slots = 2
+    q_in = [(torch.empty_like(qcs[0]), torch.empty_like(qrs[0])) for _ in range(slots)]
+    n_in = [(torch.empty_like(newc_t), torch.empty_like(newr_t)) for _ in range(slots)]
+    outs = [torch.empty_like(out) for _ in range(slots)]
+    lses = [torch.empty_like(lse) for _ in range(slots)]
+    h_outs = [torch.empty(out.shape, dtype=torch.bfloat16).pin_memory() for _ in range(slots)]
+    h_lses = [torch.empty(lse.shape, dtype=torch.float32).pin_memory() for _ in range(slots)]
+    ev_in = [torch.cuda.Event() for _ in range(slots)]
+    ev_out = [torch.cuda.Event() for _ in range(slots)]  # compute done: inputs free, outputs ready
+    ev_done = [torch.cuda.Event() for _ in range(slots)]  # read-back done: outputs free
+    for e in ev_out + ev_done:
+        e.record(stream)
 
     def e2e_step(k):
-        qcs[k].copy_(h_qc, non_blocking=True)
-        qrs[k].copy_(h_qr, non_blocking=True)
-        d_nc.copy_(h_nc, non_blocking=True)
-        d_nr.copy_(h_nr, non_blocking=True)
-        api.mla_qcache_append(desc, pools[k], table_t, hist_t, d_nc, d_nr, stream=stream)
-        api.mla_qdecode(desc, pools[k], table_t, lens_t, max_len, qcs[k], qrs[k], w.scale, out=out, lse=lse,
-                        num_splits=w.num_splits, workspace=ws, stream=stream)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
+        a = k % slots
+        hs.wait_event(ev_out[a])
+        with torch.cuda.stream(hs):
+            q_in[a][0].copy_(h_qc, non_blocking=True)
+            q_in[a][1].copy_(h_qr, non_blocking=True)
+            n_in[a][0].copy_(h_nc, non_blocking=True)
+            n_in[a][1].copy_(h_nr, non_blocking=True)
+        ev_in[a].record(hs)
+        stream.wait_event(ev_in[a])
+        stream.wait_event(ev_done[a])
+        api.mla_qcache_append(desc, pools[k % R], table_t, hist_t, n_in[a][0], n_in[a][1], stream=stream)
+        api.mla_qdecode(desc, pools[k % R], table_t, lens_t, max_len, q_in[a][0], q_in[a][1], w.scale,
+                        out=outs[a], lse=lses[a], num_splits=w.num_splits, workspace=ws, stream=stream)
+        ev_out[a].record(stream)
+        ds.wait_event(ev_out[a])
+        with torch.cuda.stream(ds):
+            h_outs[a].copy_(outs[a], non_blocking=True)
+            h_lses[a].copy_(lses[a], non_blocking=True)
+        ev_done[a].record(ds)
 
     for i in range(args.warmup):
-        e2e_step(i % R)
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    hs.wait_event(e0)
+    ds.wait_event(e0)
     for i in range(args.steps):
-        e2e_step(i % R)
+        e2e_step(i)
+    for e in ev_done:
+        stream.wait_event(e)
     e1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = e0.elapsed_time(e1) / args.steps
     if world > 1:
         ms_e2e = max_over_ranks(ms_e2e, dist, dev)
     h2d = (h_qc.numel() + h_qr.numel() + h_nc.numel() + h_nr.numel()) * 2
-    d2h = h_out.numel() * 2 + h_lse.numel() * 4
+    d2h = h_outs[0].numel() * 2 + h_lses[0].numel() * 4
 
     launches_per_step = 2 + (1 if n_split > 1 else 0)
     line = {
