@@ -18,8 +18,9 @@
 // 256-wide half of the output: O_half = 128 x 256 fp32 fits TMEM beside the
 // score buffers and the query operand.
 //
-// Precision. The dequantized values u*s+z are split into bf16 hi + bf16 lo
-// (16 significant bits together), and so are the softmax weights. Scores use
+// Precision. The dequantized values u*s+z are split into bf16 hi (the value
+// truncated to 8 significant bits) + bf16 lo (the rounded remainder), 16
+// significant bits together, and so are the softmax weights. Scores use
 // Q*C_hi + Q*C_lo (Q is exact in bf16); the output uses P_hi*C_hi + P_lo*C_hi
 // + P_hi*C_lo. All accumulation is fp32 in TMEM. This keeps the output within
 // 2e-3 of its RMS of the exact float64 result; single bf16 operands would not.
@@ -94,7 +95,7 @@ constexpr int kOffCode = kOffX + 2 * kXBuf;
 constexpr int kOffBar = kOffCode + kNS * kCodeStage + kRows * kHalfR * 2;
 constexpr int kOffQR = kOffCode + kNS * kCodeStage;  // rope part of Q: 128 rows x 32 bf16, core matrices
 constexpr int kQRBytes = kRows * kHalfR * 2;
-constexpr int kNumBars = 2 * kNS + 2 * kNC + 16 + 12;
+constexpr int kNumBars = 2 * kNS + 3 * kNC + 16 + 12;
 constexpr int kOffMisc = kOffQR + kQRBytes + kNumBars * 8;
 constexpr int kOffRed = kOffMisc + 64;  // row-pair exchange: [2 parity][2 halves][128] maxima, [2][128] sums
 constexpr int kSmemBytes = kOffRed + (2 * 2 * kRows + 2 * kRows) * 4;
@@ -112,7 +113,8 @@ struct TmapSet {
 struct Bars {
   uint64_t* code_full;   // [kNS] TMA -> dequant
   uint64_t* code_empty;  // [kNS] dequant -> TMA
-  uint64_t* c_full;      // [kNC] dequant -> MMA
+  uint64_t* c_full;      // [kNC] dequant -> MMA: channel chunks 0-15 of the stage written
+  uint64_t* c_full2;     // [kNC] dequant -> MMA: chunks 16-35 written
   uint64_t* c_empty;     // [kNC] MMA (after PV) -> dequant
   uint64_t* s_full;      // [2] MMA (QK) -> softmax
   uint64_t* s_empty;     // [2] softmax read S -> MMA
@@ -146,6 +148,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.qk_drain2 = p + 15;
   r.pair_max = p + 16;
   r.pair_sum = p + 24;
+  r.c_full2 = p + 28;
   return r;
 }
 
@@ -213,9 +216,9 @@ __device__ __forceinline__ void dequant_split8(uint32_t w, float2 s2, float2 z2,
   for (int k = 0; k < 4; ++k) {
     float2 u = __fadd2_rn(make_float2(__uint_as_float(b[2 * k]), __uint_as_float(b[2 * k + 1])), magic);
     const float2 x = __ffma2_rn(u, s2, z2);
-    __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
-    const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
-    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
+    const uint32_t ux = __float_as_uint(x.x), uy = __float_as_uint(x.y);
+    const uint32_t hw = __byte_perm(ux, uy, 0x7632);  // hi = x truncated to bf16
+    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(ux & 0xFFFF0000u), -__uint_as_float(uy & 0xFFFF0000u)));
     __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
     h[k] = hw;
     l[k] = *reinterpret_cast<uint32_t*>(&lb);
@@ -294,6 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kNC; ++i) {
       ptx::mbar_init(&bars.c_full[i], 128);
+      ptx::mbar_init(&bars.c_full2[i], 128);
       ptx::mbar_init(&bars.c_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -418,10 +422,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint64_t bs = b0 + static_cast<uint64_t>((cs * kCStage) >> 4);
         const uint32_t d = tmem + kTmemS + sb * 2 * kChunk;
+        // K-steps 0-7 read channel chunks 0-15, which the dequant warps
+        // publish first (c_full); the rest follow once c_full2 completes
 #pragma unroll
-        for (int k = 0; k < kHalfC / 16; ++k)
+        for (int k = 0; k < kHalfC / 16; ++k) {
+          if (k == kHalfC / 32) {
+            if (!ptx::mbar_wait(&bars.c_full2[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+          }
           ptx::mma_ts(d, tmem + kTmemQ + k * 8, bs + static_cast<uint64_t>((k * 2 * cstride) >> 4), idesc,
                       k > 0 ? 1u : 0u);
+        }
+        if (!ok) break;
 #pragma unroll
         for (int k = 0; k < kHalfR / 16; ++k)
           ptx::mma_ss(d, a_rope + static_cast<uint64_t>((k * 256) >> 4),
@@ -486,6 +501,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(&bars.c_full[cs]);
+      ptx::mbar_arrive(&bars.c_full2[cs]);
     }
     for (int j = 0; !kBF16 && j < n_chunks; ++j) {
       const int s = j % kNS, cs = j % kNC;
@@ -523,6 +539,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(chi + off) = hi;
           *reinterpret_cast<uint4*>(clo + off) = lo;
         }
+        if (h == 0) {  // chunks 0-15 of every token are in place: the first QK K-steps may start
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&bars.c_full[cs]);
+        }
       }
       {  // rope: 8 channels (chunk qsel of this CTA's 32)
         const uint32_t meta = *reinterpret_cast<const uint32_t*>(st + kCodeCC + kCodeRC + kCodeCM +
@@ -538,7 +558,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(clo + off) = lo;
       }
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(&bars.c_full[cs]);
+      ptx::mbar_arrive(&bars.c_full2[cs]);
       ptx::mbar_arrive(&bars.code_empty[s]);
     }
   } else if (warp >= 8) {
@@ -605,7 +625,65 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t prev[16];
     int prev_page = -1;
 
+    // Chunk jj's weight tile (my 16 tokens of this row) -> shared memory,
+    // once PV of chunk jj-2 released the buffer. False when the wait gave up.
+    auto store_weights = [&](int jj, const uint32_t (&ph)[8], const uint32_t (&pl)[8]) -> bool {
+      const int pb = jj & 1;
+      if (jj >= 2 &&
+          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, kWaitLimitNs)))
+        return false;
+      uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kc = 2 * h + kk;
+        *reinterpret_cast<uint4*>(pt + kc * 128) = make_uint4(ph[4 * kk], ph[4 * kk + 1], ph[4 * kk + 2], ph[4 * kk + 3]);
+        *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
+            make_uint4(pl[4 * kk], pl[4 * kk + 1], pl[4 * kk + 2], pl[4 * kk + 3]);
+      }
+      return true;
+    };
+    // The O rescale a grown maximum needs, then the release of chunk jj's
+    // weight tile to the PV issuer. `fence`: the tile's stores still need the
+    // generic -> async proxy fence (a later fence of this thread covers them
+    // too). False when a wait gave up.
+    auto release_weights = [&](int jj, float alpha, bool rescale, bool fence) -> bool {
+      // rescale my half of this row of O in TMEM (warp-collective: lanes that
+      // do not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
+      if (__any_sync(kFull, rescale && o_live)) {
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
+                                              kWaitLimitNs)))
+          return false;
+        ptx::tc_fence_after();
+        const float f = (rescale && o_live) ? alpha : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < kHalfC / 64; ++c) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+          ptx::tmem_st32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
+        }
+        ptx::tmem_st_wait();
+      }
+      o_live = true;
+      if (fence) ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars.p_full[jj & 1]);
+      return true;
+    };
+
+    // Step j: the scores and weight tile of chunk j-1 (it needs the peer's
+    // partial, sent one step earlier), then the read and send of this CTA's
+    // partial of chunk j. The quantized path releases chunk j-1's tile to PV
+    // only after the send (whose proxy fence then covers the tile too), so
+    // the release and any O rescale fill the time the copy is in flight; the
+    // BF16 path releases it first, since its operand stages wait on PV and
+    // then on HBM.
     for (int j = 0; j <= n_chunks && ok; ++j) {
+      uint32_t ph[8], pl[8];
+      float alpha = 1.0f;
+      bool rescale = false;
       if (j >= 1) {
         const int jj = j - 1, pb = jj & 1;
         const int t0 = t_begin + jj * kChunk;
@@ -650,8 +728,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         const float mx = fmaxf(mt[0], red_max[(pb * 2 + (h ^ 1)) * kRows + i]);
-        float alpha = 1.0f;
-        bool rescale = false;
         if (mx > -CUDART_INF_F) {
           if (m_used == -CUDART_INF_F) {
             m_used = mx;
@@ -664,16 +740,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // p = 2^(s - m); rows that have seen no key use m = 0, so every p is 0
         const float m_eff = (m_used == -CUDART_INF_F) ? 0.0f : m_used;
         const float2 negm = make_float2(-m_eff, -m_eff);
-        uint32_t ph[8], pl[8];
         float2 ps[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float2 d = __fadd2_rn(sp[k], negm);
           const float2 pk = make_float2(ex2_approx(d.x), ex2_approx(d.y));
           ps[k] = pk;
-          __nv_bfloat162 hb = __floats2bfloat162_rn(pk.x, pk.y);
-          const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
-          const float2 r = __fadd2_rn(pk, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
+          // hi = p truncated to bf16 (a byte permute), lo = bf16(p - hi)
+          const uint32_t ux = __float_as_uint(pk.x), uy = __float_as_uint(pk.y);
+          const uint32_t hw = __byte_perm(ux, uy, 0x7632);
+          const float2 r = __fadd2_rn(pk, make_float2(-__uint_as_float(ux & 0xFFFF0000u), -__uint_as_float(uy & 0xFFFF0000u)));
           __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
           ph[k] = hw;
           pl[k] = *reinterpret_cast<uint32_t*>(&lb);
@@ -684,47 +760,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int k = 0; k < w; ++k) ps[k] = __fadd2_rn(ps[k], ps[k + w]);
         l_sum = l_sum * alpha + (ps[0].x + ps[0].y);
 
-        // P tile (my 16 tokens of this row) -> smem, once PV of chunk jj-2 released the buffer
-        if (jj >= 2 &&
-            !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+      }
+      if (j >= 1 && !store_weights(j - 1, ph, pl)) {
+        ok = false;
+        break;
+      }
+      if constexpr (kBF16) {  // operands arrive straight from HBM: release PV as early as possible
+        if (j >= 1 && !release_weights(j - 1, alpha, rescale, true)) {
           ok = false;
           break;
         }
-        uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int kc = 2 * h + kk;
-          *reinterpret_cast<uint4*>(pt + kc * 128) =
-              make_uint4(ph[4 * kk], ph[4 * kk + 1], ph[4 * kk + 2], ph[4 * kk + 3]);
-          *reinterpret_cast<uint4*>(pt + kPTile + kc * 128) =
-              make_uint4(pl[4 * kk], pl[4 * kk + 1], pl[4 * kk + 2], pl[4 * kk + 3]);
-        }
-
-        // rescale my half of this row of O in TMEM (warp-collective: lanes that
-        // do not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
-        if (__any_sync(kFull, rescale && o_live)) {
-          if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
-                                                kWaitLimitNs))) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          const float f = (rescale && o_live) ? alpha : 1.0f;
-#pragma unroll 1
-          for (int c = 0; c < kHalfC / 64; ++c) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-            ptx::tmem_st32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
-          }
-          ptx::tmem_st_wait();
-        }
-        o_live = true;
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars.p_full[pb]);
       }
       uint32_t cur[16];
       int cur_page = -1;
@@ -739,12 +784,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + 16 * h, cur);
-        if (n_terms_qk == 2) {  // add the C_lo half of the score tile
-          uint32_t lo[16];
-          ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + kChunk + 16 * h, lo);
-          ptx::tmem_ld_wait();
+        if (n_terms_qk == 2) {  // add the C_lo half of the score tile, 8 columns at a time
 #pragma unroll
-          for (int k = 0; k < 16; ++k) cur[k] = __float_as_uint(__uint_as_float(cur[k]) + __uint_as_float(lo[k]));
+          for (int g = 0; g < 2; ++g) {
+            uint32_t lo[8];
+            ptx::tmem_ld8(lane_base + kTmemS + sb * 2 * kChunk + kChunk + 16 * h + 8 * g, lo);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              cur[8 * g + k] = __float_as_uint(__uint_as_float(cur[8 * g + k]) + __uint_as_float(lo[k]));
+          }
         }
         ptx::tmem_ld_wait();
         ptx::tc_fence_before();
@@ -764,6 +813,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0)
           ptx::bulk_copy_to_peer(xbuf_peer + sb * kXBuf + blk, smem + kOffX + (sb ^ 1) * kXBuf + blk, kXWarpBlock,
                                  xfull_peer + sb * 8);
+      }
+      if constexpr (!kBF16) {
+        if (j >= 1 && !release_weights(j - 1, alpha, rescale, j == n_chunks)) {
+          ok = false;
+          break;
+        }
       }
 #pragma unroll
       for (int k = 0; k < 16; ++k) prev[k] = cur[k];
