@@ -77,10 +77,12 @@ constexpr int kCLoOff = 512;
 constexpr int kCStage = kKChunks * kCChunkStride;
 constexpr int kBfChunkStride = 512;  // bf16 cache: C only, [chunk][token group][8 rows x 16 B]
 constexpr int kPTile = (kRows / 8) * 4 * 128;      // 8 KB: 16 row groups x 4 token groups x 128 B
-// Score-exchange slot: [column half h][row][20 floats] (16 scores + 4 pad, a
-// bank-conflict-free stride for 16-byte accesses). The 32 rows one softmax warp
-// owns in one half are a contiguous 2560-byte block, sent as one bulk copy.
-constexpr int kXRowBytes = 80;
+// Score-exchange slot: [column half h][row][16 floats]. The four 16-byte
+// pieces of row i are stored in the order k ^ ((i >> 1) & 3), so that eight
+// consecutive rows' 16-byte accesses cover all 32 banks. The 32 rows one
+// softmax warp owns in one half are a contiguous 2048-byte block, sent as one
+// bulk copy (the copy moves bytes, so both sides see the same order).
+constexpr int kXRowBytes = 64;
 constexpr int kXWarpBlock = 32 * kXRowBytes;
 constexpr int kXHalf = kRows * kXRowBytes;
 constexpr int kXBuf = 2 * kXHalf;
@@ -697,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float2 sp[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float4 pv = xr[k];
+          const float4 pv = xr[k ^ ((i >> 1) & 3)];
           sp[2 * k] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k]), __uint_as_float(prev[4 * k + 1])),
                                             make_float2(pv.x, pv.y)), sc2);
           sp[2 * k + 1] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k + 2]),
@@ -806,7 +808,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint8_t* stage = smem + kOffX + (sb ^ 1) * kXBuf + h * kXHalf + i * kXRowBytes;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(stage + 16 * k) = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
+          *reinterpret_cast<uint4*>(stage + 16 * (k ^ ((i >> 1) & 3))) = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
         ptx::fence_proxy_async_smem();
         __syncwarp();
         if (i == 0 && h == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kXBuf);
