@@ -10,6 +10,7 @@
 // bit for bit.
 #include "mla_common.cuh"
 #include "mla_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 
@@ -39,6 +40,7 @@ qcache_append_kernel(uint8_t* __restrict__ pool, int num_pages, const int32_t* _
                      const __nv_bfloat16* __restrict__ src_pool, int src_num_pages,
                      const int32_t* __restrict__ src_pages, int n_tokens, int n_new, int* status) {
   using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
+  ptx::griddep_launch_dependents();  // a decode launched as a programmatic dependent may be scheduled now
   const int lane = threadIdx.x & 31;
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (tok >= n_tokens) return;
@@ -146,6 +148,7 @@ bf16cache_append_kernel(__nv_bfloat16* __restrict__ pool, int num_pages, const i
                         int max_pages, const int32_t* __restrict__ lens_before,
                         const __nv_bfloat16* __restrict__ c_new, const __nv_bfloat16* __restrict__ kr_new,
                         int n_tokens, int n_new, int* status) {
+  ptx::griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (tok >= n_tokens) return;

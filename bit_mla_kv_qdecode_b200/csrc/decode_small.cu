@@ -123,6 +123,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
   using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
   using Lo = Layout<G>;
   static_assert(BITS_C == 4 && G_C == 64 && BITS_R == 4 && G_R == 64, "INT4 g64 content and RoPE");
+  // launched as a programmatic dependent: wait for the previous grid before any read
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lo::kOffBar);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lo::kOffMisc);
@@ -490,8 +493,8 @@ cudaError_t launch_t(const DecodeLaunch& L) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lo::kBytes);
   if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(L);
-  kern<<<static_cast<unsigned>(L.B * L.n_split), kThreads, Lo::kBytes, L.stream>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3(static_cast<unsigned>(L.B * L.n_split)), dim3(kThreads), Lo::kBytes, L.stream,
+                          a);
 }
 
 }  // namespace small

@@ -243,6 +243,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_tc_kernel(const DecodeArgs a, const __grid_constant__ TmapSet tm, int row_tiles, int n_terms_qk,
                      int n_terms_pv) {
   using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
+  // launched as a programmatic dependent: wait for the previous grid (e.g. the
+  // cache append) before any read, then let the combine be scheduled
+  ptx::griddep_wait();
+  ptx::griddep_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Bars bars = carve_bars(smem);
@@ -979,8 +983,8 @@ cudaError_t launch_t(const DecodeLaunch& L) {
   const bool fast = (L.flags & MLA_DECODE_FAST_UNCOMPENSATED) != 0;
   const int terms_qk = (kBF16 || fast) ? 1 : 2;
   const int terms_pv = fast ? 1 : (kBF16 ? 2 : 3);
-  kern<<<static_cast<unsigned>(units * 2), kThreads, kSmemAlloc, L.stream>>>(a, tm, row_tiles, terms_qk, terms_pv);
-  return cudaGetLastError();
+  return launch_dependent(kern, dim3(static_cast<unsigned>(units * 2)), dim3(kThreads), kSmemAlloc, L.stream, a, tm,
+                          row_tiles, terms_qk, terms_pv);
 }
 
 }  // namespace tc

@@ -161,6 +161,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Block until the grids this one depends on (programmatic stream
+// serialization) have completed and their writes are visible. A no-op when
+// the grid was launched without that attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream, when launched as a programmatic
+// dependent, to be scheduled before this one finishes (it still waits for
+// this grid's completion before it reads anything).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
   asm volatile(
