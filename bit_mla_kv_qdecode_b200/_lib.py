@@ -52,6 +52,9 @@ SIGNATURES = {
     "mla_qdecode": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void, _c_int, _c_int,
                              _c_int, _c_float, _c_int, _c_void, _c_size, _c_void, _c_int, _c_void, _c_uint,
                              _c_void]),
+    "mla_qdecode_fused_append": (_c_int, [_P, _c_void, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void, _c_int,
+                                          _c_void, _c_void, _c_int, _c_int, _c_int, _c_float, _c_int, _c_void,
+                                          _c_size, _c_void, _c_int, _c_void, _c_uint, _c_void]),
     "mla_decode_bf16": (_c_int, [_c_void, _c_int, _c_int, _c_void, _c_int, _c_void, _c_int, _c_void, _c_void,
                                  _c_int, _c_int, _c_int, _c_float, _c_int, _c_void, _c_size, _c_void, _c_int,
                                  _c_void, _c_uint, _c_void]),

@@ -135,6 +135,24 @@ def mla_qdecode_noalloc(desc, pool, block_table, seq_lens, max_seq_len, q_c, q_r
     return out, lse
 
 
+def mla_qdecode_fused_append(desc, pool, block_table, seq_lens, max_seq_len, c_new, kr_new, q_c, q_r, scale, *,
+                             out=None, out_dtype=torch.bfloat16, lse=None, num_splits=0, workspace=None, flags=0,
+                             stream=None):
+    """Append the step's new tokens (c_new [B, n, 512], kr_new [B, n, 64]; seq_lens count them) and
+    decode, in one call. Returns (out, lse). See include/mla_qcache.h for the contract."""
+    (B, s_q, H), qc, qr, out, po, pl, pw, nw, f32, _ = _decode_io(
+        q_c, q_r, out, out_dtype, lse, workspace, max_seq_len, num_splits)
+    if seq_lens.shape[0] != B or c_new.shape[0] != B:
+        raise ValueError("seq_lens and c_new must have one entry per request")
+    n = c_new.shape[1]
+    check("mla_qdecode_fused_append", _lib.load().mla_qdecode_fused_append(
+        ctypes.byref(desc), _need(pool, "pool", torch.uint8), _need(block_table, "block_table", torch.int32),
+        block_table.shape[1], _need(seq_lens, "seq_lens", torch.int32), int(max_seq_len),
+        _need(c_new, "c_new", torch.bfloat16, (B, n, D_C)), _need(kr_new, "kr_new", torch.bfloat16, (B, n, D_R)), n,
+        qc, qr, B, s_q, H, float(scale), int(num_splits), pw, nw, po, f32, pl, int(flags), _stream(stream)))
+    return out, lse
+
+
 def mla_decode_bf16(pool, block_table, seq_lens, max_seq_len, q_c, q_r, scale, *, out=None,
                     out_dtype=torch.bfloat16, lse=None, num_splits=0, workspace=None, flags=0, stream=None):
     (B, s_q, H), qc, qr, out, po, pl, pw, nw, f32, _ = _decode_io(

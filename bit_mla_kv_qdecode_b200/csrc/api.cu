@@ -135,6 +135,10 @@ struct DecodeCommon {
   float* lse;
   unsigned flags;
   cudaStream_t stream;
+  // fused append (quantized cache): new tokens, the last n_new of seq_lens[b]
+  const void* c_new;
+  const void* kr_new;
+  int n_new;
 };
 
 mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_desc* desc) {
@@ -143,6 +147,9 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   if (c.out_dtype != 0 && c.out_dtype != 1) return MLA_ERR_INVALID_ARG;
   if (!isfinite(c.scale)) return MLA_ERR_INVALID_ARG;
   if (c.flags & ~(MLA_DECODE_FORCE_SIMT | MLA_DECODE_FAST_UNCOMPENSATED)) return MLA_ERR_INVALID_ARG;
+  if (c.n_new < 0 || (c.n_new > 0 && (!quantized || !c.c_new || !c.kr_new))) return MLA_ERR_INVALID_ARG;
+  if (c.n_new > 0 && (!aligned(c.c_new, 16) || !aligned(c.kr_new, 16) || !c.pool)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<long>(c.B) * c.n_new > (1L << 26)) return MLA_ERR_UNSUPPORTED;
   if (c.B == 0) return MLA_OK;
   if (c.B > 65535 || static_cast<long>(c.s_q) * c.H > (1 << 20)) return MLA_ERR_UNSUPPORTED;
   if (!c.block_table || !c.seq_lens || !c.q_c || !c.q_r || !c.out) return MLA_ERR_INVALID_ARG;
@@ -197,16 +204,37 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   L.status = status;
   L.stream = c.stream;
 
+  // A fused append runs inside the tensor-core kernel; the other kernels get
+  // the append kernel launched first (lengths here already count the new tokens).
+  auto append_first = [&]() -> cudaError_t {
+    mla::AppendLaunch A{const_cast<void*>(c.pool), c.num_pages, c.block_table, c.max_pages_per_seq, c.seq_lens,
+                        c.c_new, c.kr_new, c.B, c.n_new, L.bits_c, L.group_c, L.bits_r, L.group_r,
+                        nullptr, 0, nullptr, status, c.stream, -c.n_new};
+    return mla::launch_qcache_append(A);
+  };
   cudaError_t e = cudaErrorNotSupported;
   if (!(c.flags & MLA_DECODE_FORCE_SIMT)) {
+    if (c.n_new > 0 && mla::decode_small_supported(L)) {
+      if (append_first() != cudaSuccess) return MLA_ERR_CUDA;
+    } else if (c.n_new > 0) {
+      L.c_new = c.c_new;
+      L.kr_new = c.kr_new;
+      L.n_new = c.n_new;
+    }
     e = mla::launch_decode_small(L);
     if (e == cudaErrorNotSupported) {
       cudaGetLastError();
-      e = mla::launch_decode_tc(L);
+      e = mla::launch_decode_tc(L);  // returns NotSupported before launching anything
     }
   }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
+    if (L.n_new > 0) {  // the tensor-core kernel did not take the fused append
+      L.n_new = 0;
+      if (append_first() != cudaSuccess) return MLA_ERR_CUDA;
+    } else if (c.n_new > 0 && (c.flags & MLA_DECODE_FORCE_SIMT)) {
+      if (append_first() != cudaSuccess) return MLA_ERR_CUDA;
+    }
     e = mla::launch_decode_simt(L);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
@@ -340,6 +368,21 @@ mla_status mla_qdecode(const mla_qcache_desc* desc, const void* pool, const int3
   DecodeCommon c{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens, max_seq_len, q_c, q_r,
                  B, s_q, H, scale, num_splits, workspace, workspace_bytes, out, out_dtype, lse, flags,
                  reinterpret_cast<cudaStream_t>(stream)};
+  return run_decode(c, true, desc);
+}
+
+mla_status mla_qdecode_fused_append(const mla_qcache_desc* desc, void* pool, const int32_t* block_table,
+                                    int max_pages_per_seq, const int32_t* seq_lens, int max_seq_len,
+                                    const void* c_new, const void* kr_new, int n_new, const void* q_c,
+                                    const void* q_r, int B, int s_q, int H, float scale, int num_splits,
+                                    void* workspace, size_t workspace_bytes, void* out, int out_dtype, float* lse,
+                                    unsigned flags, mla_stream_t stream) {
+  const mla_status st = mla_qcache_check_desc(desc);
+  if (st != MLA_OK) return st;
+  if (n_new < 0 || (n_new > 0 && !pool)) return MLA_ERR_INVALID_ARG;
+  DecodeCommon c{pool, desc->num_pages, block_table, max_pages_per_seq, seq_lens, max_seq_len, q_c, q_r,
+                 B, s_q, H, scale, num_splits, workspace, workspace_bytes, out, out_dtype, lse, flags,
+                 reinterpret_cast<cudaStream_t>(stream), c_new, kr_new, n_new};
   return run_decode(c, true, desc);
 }
 

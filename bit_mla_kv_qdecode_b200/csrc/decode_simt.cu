@@ -335,6 +335,9 @@ DecodeArgs make_decode_args(const DecodeLaunch& L) {
   a.chunk_pages = L.chunk_pages;
   a.out_f32 = L.out_f32;
   a.scale_log2 = L.scale * kLog2e;
+  a.c_new = static_cast<const __nv_bfloat16*>(L.c_new);
+  a.kr_new = static_cast<const __nv_bfloat16*>(L.kr_new);
+  a.n_new = L.n_new;
   return a;
 }
 

@@ -499,10 +499,14 @@ cudaError_t launch_t(const DecodeLaunch& L) {
 
 }  // namespace small
 
+bool decode_small_supported(const DecodeLaunch& L) {
+  return L.quantized && L.s_q * L.H <= small::kRows && L.num_pages >= 1 && L.bits_c == 4 && L.group_c == 64 &&
+         L.bits_r == 4 && L.group_r == 64;
+}
+
 cudaError_t launch_decode_small(const DecodeLaunch& L) {
-  if (!L.quantized || L.s_q * L.H > small::kRows || L.num_pages < 1) return cudaErrorNotSupported;
-  if (L.bits_c == 4 && L.group_c == 64 && L.bits_r == 4 && L.group_r == 64) return small::launch_t<4, 64, 4, 64>(L);
-  return cudaErrorNotSupported;
+  if (!decode_small_supported(L)) return cudaErrorNotSupported;
+  return small::launch_t<4, 64, 4, 64>(L);
 }
 
 }  // namespace mla

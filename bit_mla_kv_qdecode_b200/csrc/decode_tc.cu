@@ -42,6 +42,7 @@
 
 #include <mutex>
 
+#include "append_token.cuh"
 #include "mla_common.cuh"
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
@@ -273,6 +274,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int row0 = rt * kRows;
 
   if (n_chunks == 0) {  // no keys: o = 0, lse = -inf (single-split plans write the output)
+    if (a.n_new > T && tid == 0 && crank == 0) record_error(a.status, MLA_ERR_INVALID_ARG);
     if (tid < kRows) {
       const int row = row0 + tid;
       if (row < a.rows) {
@@ -331,9 +333,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptx::tmem_alloc(tmem_slot, kTmemCols);
     ptx::tmem_relinquish();
   }
+  if constexpr (!kBF16) {
+    // Fused append: the step's n_new new tokens are the last n_new of the T
+    // positions. CTA 0 of the pair quantizes those inside this unit's key
+    // range into the pool (one warp per token, the same writer as the append
+    // kernel) before either CTA loads a page; the proxy fence and the cluster
+    // barrier below order those writes before the TMA reads. Row tiles of one
+    // request write identical bytes.
+    if (a.n_new > 0 && crank == 0 && warp >= 8) {
+      if (T < a.n_new) {
+        if (tid == 256) record_error(a.status, MLA_ERR_INVALID_ARG);
+      } else {
+        const int t_new = T - a.n_new;
+        for (int t = max(t_new, t_begin) + (warp - 8); t < t_end; t += 8) {
+          const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t);
+          if (page < 0) {
+            if (lane == 0) record_error(a.status, MLA_ERR_INVALID_ARG);
+            continue;
+          }
+          const size_t src = static_cast<size_t>(b) * a.n_new + (t - t_new);
+          quantize_token_warp<BITS_C, G_C, BITS_R, G_R>(
+              const_cast<uint8_t*>(a.pool) + static_cast<size_t>(page) * G::kPageBytes, t % kPage,
+              a.c_new + src * kDc, a.kr_new + src * kDr, lane);
+        }
+        ptx::fence_proxy_async_global();
+      }
+    }
+  }
   ptx::tc_fence_before();
   __syncthreads();
-  ptx::cluster_sync();  // peer barriers are initialised before any remote arrive
+  ptx::cluster_sync();  // peer barriers are initialised before any remote arrive; fused-append writes are visible
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -368,6 +397,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int cs = 0; cs < kNC; ++cs)
         if (issued[cs] > 0) ptx::mbar_wait(&bars.code_full[cs], ((issued[cs] - 1) / kNC) & 1, nullptr, kWaitLimitNs);
     } else if (lane == 0) {
+      if (a.n_new > 0) ptx::fence_proxy_async_global();  // the fused append's writes precede these TMA reads
       const uint32_t bytes = kChunk * (G::kRowC / 2) + kChunk * G::kRowR + kChunk * (G::kGroupsC * 2) +
                              kChunk * G::kGroupsR * 4;
       int issued[kNS];

@@ -85,6 +85,9 @@ struct DecodeArgs {
   int n_split, chunk_pages;
   int out_f32;
   float scale_log2;          // softmax scale * log2(e)
+  const __nv_bfloat16* c_new;   // fused append: [B, n_new, 512] (tensor-core kernel only)
+  const __nv_bfloat16* kr_new;  // [B, n_new, 64]
+  int n_new;                    // 0: no fused append
 };
 
 // Keys visible to flattened row r = i*H + h of a request holding T keys.

@@ -44,6 +44,9 @@ struct AppendLaunch {
   const int32_t* src_pages;
   int* status;
   cudaStream_t stream;
+  // position of new token j of request b: lens_before[b] + lens_offset + j
+  // (-n_new when the lengths passed already count the new tokens)
+  int lens_offset;
 };
 
 cudaError_t launch_qcache_append(const AppendLaunch& L);
@@ -72,6 +75,12 @@ struct DecodeLaunch {
   unsigned flags;
   int* status;
   cudaStream_t stream;
+  // fused append (tensor-core kernel only): bf16 c_new [B, n_new, 512] and
+  // kr_new [B, n_new, 64] are the last n_new of seq_lens[b] positions; each
+  // unit quantizes those in its key range into the pool before reading it
+  const void* c_new;
+  const void* kr_new;
+  int n_new;
 };
 
 struct DecodeArgs;
@@ -89,6 +98,7 @@ cudaError_t launch_decode_tc(const DecodeLaunch& L);
 // Warp-level MMA kernel for s_q * H <= 16 rows (INT4 g64 content and RoPE);
 // cudaErrorNotSupported for other shapes and formats.
 cudaError_t launch_decode_small(const DecodeLaunch& L);
+bool decode_small_supported(const DecodeLaunch& L);
 // Query rows up to which a decode unit is one CTA of the small-row kernel.
 constexpr int kSmallRows = 16;
 

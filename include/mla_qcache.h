@@ -202,6 +202,36 @@ mla_status mla_qdecode(const mla_qcache_desc* desc, const void* pool,
                        void* out, int out_dtype, float* lse,
                        unsigned flags, mla_stream_t stream);
 
+/* One decode step of a speculative-verify / multi-token-prediction loop:
+ * the cache append of the step's n_new new tokens followed by mla_qdecode,
+ * with the append fused into the decode kernel where the tensor-core kernel
+ * runs (each work unit quantizes the new tokens inside its key range into the
+ * pool, then reads them back through TMA), which saves the append launch and
+ * its latency. Results and pool bytes are those of mla_qcache_append
+ * (seq_lens_before = seq_lens - n_new) followed by mla_qdecode; where the
+ * fused form does not apply (s_q*H <= 16, MLA_DECODE_FORCE_SIMT) the library
+ * launches the append kernel and then the decode itself.
+ * (QuantMLA abstract: tokens are quantized as they are written; the
+ * workload's verify step appends s_q tokens per request before the decode.)
+ *   seq_lens      device int32 [B]: lengths AFTER the append; the new tokens
+ *                 are positions [seq_lens[b] - n_new, seq_lens[b]). A length
+ *                 below n_new is flagged in the device status word and its
+ *                 tokens are not written.
+ *   c_new, kr_new device bf16 [B, n_new, d_c] and [B, n_new, d_r], 16-byte
+ *                 aligned, finite, |x| <= 65504.
+ *   n_new         >= 0 (0 makes this exactly mla_qdecode).
+ *   pool          device, written in place (the new tokens' slots only).
+ *   other arguments as for mla_qdecode. */
+mla_status mla_qdecode_fused_append(const mla_qcache_desc* desc, void* pool,
+                                    const int32_t* block_table, int max_pages_per_seq,
+                                    const int32_t* seq_lens, int max_seq_len,
+                                    const void* c_new, const void* kr_new, int n_new,
+                                    const void* q_c, const void* q_r,
+                                    int B, int s_q, int H, float scale, int num_splits,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* out, int out_dtype, float* lse,
+                                    unsigned flags, mla_stream_t stream);
+
 /* The same decode over the unquantized comparison cache (pool as for
  * mla_bf16cache_append: device bf16 [num_pages, page_size, d_c + d_r]). */
 mla_status mla_decode_bf16(const void* pool, int num_pages, int page_size,

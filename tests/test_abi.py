@@ -149,3 +149,19 @@ def test_cache_capacity_closed_forms(lib):
     assert api.mla_cache_bytes_per_request(d44, -1) == 0
     assert api.mla_cache_bytes_per_request(None, T, 64, 0) == 0
     assert api.mla_cache_max_requests(d44, 0, budget) == -1
+
+
+def test_fused_append_argument_errors(lib):
+    E = _lib
+    d = ctypes.byref(_lib.make_desc(4, 64, num_pages=8))
+
+    def call(pool=FAKE, cn=FAKE, kn=FAKE, n=1, B=2, flags=0):
+        return lib.mla_qdecode_fused_append(d, pool, FAKE, 4, FAKE, 256, cn, kn, n, FAKE, FAKE, B, 1, 128, 0.1, 1,
+                                            None, 0, FAKE, 0, None, flags, None)
+
+    assert call(n=-1) == E.MLA_ERR_INVALID_ARG
+    assert call(cn=None) == E.MLA_ERR_INVALID_ARG
+    assert call(kn=FAKE + 8) == E.MLA_ERR_INVALID_ARG                 # not 16-byte aligned
+    assert call(pool=None) == E.MLA_ERR_INVALID_ARG
+    assert call(B=0) == E.MLA_OK
+    assert call(B=0, n=0, cn=None, kn=None) == E.MLA_OK
