@@ -56,26 +56,34 @@ struct SplitPlan {
   int chunk_pages;
 };
 
-// Split each request's pages into n page-aligned chunks. An explicit request
-// is honoured (capped at the page count). The automatic choice models the
-// decode time of the longest request as waves(n) * (pages / n), where a wave
-// is one work unit (128 query rows of one request and one split) on each
-// 2-CTA cluster slot -- or, for at most 16 query rows, one request and split
-// on each of two CTA slots per SM (the small-row kernel) -- and picks the
-// smallest n within 3% of the best, with chunks of at least 4 pages.
+// Split each request's pages into n page-aligned chunks. No chunk holds more
+// than kMaxChunkPages pages: the tensor cores' fp32 accumulation loses
+// accuracy in proportion to the keys one accumulator sums (measured on B200
+// at about 5e-8 x RMS per key), so 8,192 keys keep the output within about
+// 4.5e-4 x RMS of exact, a fourfold margin on the stated bound. An explicit
+// request is honoured (capped at the page count) when it meets that limit and
+// raised to it otherwise. The automatic choice models the decode time of the
+// longest request as waves(n) * (pages / n), where a wave is one work unit
+// (128 query rows of one request and one split) on each 2-CTA cluster slot --
+// or, for at most 16 query rows, one request and split on each of two CTA
+// slots per SM (the small-row kernel) -- and picks the smallest n within 3% of
+// the best, with chunks of at least 4 pages.
+constexpr int kMaxChunkPages = 128;
+
 SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
   const int pages = std::max(1, (max_seq_len + mla::kPage - 1) / mla::kPage);
+  const int n_min = (pages + kMaxChunkPages - 1) / kMaxChunkPages;
   int n;
   if (requested > 0) {
-    n = std::min(requested, pages);
+    n = std::max(std::min(requested, pages), n_min);
   } else {
     const bool small = static_cast<long>(s_q) * H <= mla::kSmallRows;
     const long units = static_cast<long>(std::max(B, 1)) * (small ? 1 : (static_cast<long>(s_q) * H + 127) / 128);
     const long slots = std::max(1, small ? 2 * device_sm_count() : device_sm_count() / 2);
-    const int n_max = std::max(1, std::min(pages / 4, 64));
+    const int n_max = std::max(n_min, std::min(pages / 4, 64));
     double best = 1e30;
-    n = 1;
-    for (int c = 1; c <= n_max; ++c) {
+    n = n_min;
+    for (int c = n_min; c <= n_max; ++c) {
       const long waves = (units * c + slots - 1) / slots;
       const double cost = static_cast<double>(waves) * ((pages + c - 1) / c) + 2.0 * waves;  // + per-unit overhead
       if (cost < best * 0.97) {

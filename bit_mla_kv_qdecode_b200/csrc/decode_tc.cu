@@ -18,9 +18,11 @@
 // 256-wide half of the output: O_half = 128 x 256 fp32 fits TMEM beside the
 // score buffers and the query operand.
 //
-// Precision. The dequantized values u*s+z are split into bf16 hi (the value
-// truncated to 8 significant bits) + bf16 lo (the rounded remainder), 16
-// significant bits together, and so are the softmax weights. Scores use
+// Precision. The dequantized values u*s+z are split into bf16 hi + bf16 lo
+// (both rounded to nearest; 16 significant bits together), and so are the
+// softmax weights. Rounding, not truncating, the hi part keeps the dropped
+// P_lo*C_lo term zero-mean; with truncated hi parts it is biased and the
+// output error grew with the sequence length (measured). Scores use
 // Q*C_hi + Q*C_lo (Q is exact in bf16); the output uses P_hi*C_hi + P_lo*C_hi
 // + P_hi*C_lo. All accumulation is fp32 in TMEM. This keeps the output within
 // 2e-3 of its RMS of the exact float64 result; single bf16 operands would not.
@@ -219,9 +221,9 @@ __device__ __forceinline__ void dequant_split8(uint32_t w, float2 s2, float2 z2,
   for (int k = 0; k < 4; ++k) {
     float2 u = __fadd2_rn(make_float2(__uint_as_float(b[2 * k]), __uint_as_float(b[2 * k + 1])), magic);
     const float2 x = __ffma2_rn(u, s2, z2);
-    const uint32_t ux = __float_as_uint(x.x), uy = __float_as_uint(x.y);
-    const uint32_t hw = __byte_perm(ux, uy, 0x7632);  // hi = x truncated to bf16
-    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(ux & 0xFFFF0000u), -__uint_as_float(uy & 0xFFFF0000u)));
+    __nv_bfloat162 hb = __floats2bfloat162_rn(x.x, x.y);
+    const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
     __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
     h[k] = hw;
     l[k] = *reinterpret_cast<uint32_t*>(&lb);
@@ -782,10 +784,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const float2 d = __fadd2_rn(sp[k], negm);
           const float2 pk = make_float2(ex2_approx(d.x), ex2_approx(d.y));
           ps[k] = pk;
-          // hi = p truncated to bf16 (a byte permute), lo = bf16(p - hi)
-          const uint32_t ux = __float_as_uint(pk.x), uy = __float_as_uint(pk.y);
-          const uint32_t hw = __byte_perm(ux, uy, 0x7632);
-          const float2 r = __fadd2_rn(pk, make_float2(-__uint_as_float(ux & 0xFFFF0000u), -__uint_as_float(uy & 0xFFFF0000u)));
+          __nv_bfloat162 hb = __floats2bfloat162_rn(pk.x, pk.y);
+          const uint32_t hw = *reinterpret_cast<uint32_t*>(&hb);
+          const float2 r = __fadd2_rn(pk, make_float2(-__uint_as_float(hw << 16), -__uint_as_float(hw & 0xFFFF0000u)));
           __nv_bfloat162 lb = __floats2bfloat162_rn(r.x, r.y);
           ph[k] = hw;
           pl[k] = *reinterpret_cast<uint32_t*>(&lb);

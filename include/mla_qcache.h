@@ -185,6 +185,9 @@ size_t mla_decode_workspace_bytes(int B, int s_q, int H, int max_seq_len, int nu
  *   scale         softmax scale applied to the sum of both dot products.
  *   num_splits    0 = library choice; > 0 = split each request's keys into
  *                 that many page-aligned chunks merged by a combine kernel.
+ *                 Either way no chunk holds more than 8,192 keys (the count
+ *                 is raised when needed): the tensor cores' fp32 accumulation
+ *                 loses accuracy in proportion to the keys one chunk sums.
  *   workspace     device, >= mla_decode_workspace_bytes(...) bytes, 256-byte
  *                 aligned (may be NULL when that size is 0). Caller-owned
  *                 scratch; contents need no initialisation.

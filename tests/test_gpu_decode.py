@@ -153,3 +153,16 @@ def test_full_size_workloads(idx):
         out, lse = run_decode(case, pool_b, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16,
                               quantized=False)
         check(case, out, lse, FULL[idx], quantized=False, bf16_out=True)
+
+
+def test_long_request_chunk_cap():
+    # 32,768 keys asked for as one split: the library raises the split count so
+    # that no accumulator sums more than 8,192 keys, which keeps the error well
+    # inside the bound (one 32K-key chunk measured 1.75e-3 x RMS)
+    w = synth.workload(3).scaled(B=1, t_lo=32768, t_hi=32768)
+    assert api.mla_decode_num_splits(1, 1, 128, 32768, 1) == 4
+    case = mc.make_case(w)
+    pool, table_t = mc.fill_pool(case)
+    out, lse = run_decode(case, pool, table_t, num_splits=1)
+    err = check(case, out, lse, [0])
+    assert err < 1e-3, err
