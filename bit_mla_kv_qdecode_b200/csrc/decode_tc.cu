@@ -104,6 +104,11 @@ constexpr int kNumBars = 2 * kNS + 3 * kNC + 16 + 12;
 constexpr int kOffMisc = kOffQR + kQRBytes + kNumBars * 8;
 constexpr int kOffRed = kOffMisc + 64;  // row-pair exchange: [2 parity][2 halves][128] maxima, [2][128] sums
 constexpr int kSmemBytes = kOffRed + (2 * 2 * kRows + 2 * kRows) * 4;
+// Epilogue staging of the output rows, over the operand stages and weight tiles
+// (free once every MMA has completed): [row][2 halves x 512 B] + 16 B of pad,
+// so that the 16-byte stores of eight consecutive rows hit distinct banks.
+constexpr int kEpiRow = 2 * 512 + 16;
+static_assert(kOffC + kRows * kEpiRow <= kOffX, "epilogue staging fits the operand and weight-tile stages");
 constexpr int kSmemAlloc = kSmemBytes + 1024;      // slack to align the base to 1024
 static_assert(kOffCode % 1024 == 0 && kCodeStage % 1024 == 0, "TMA swizzle needs 1024-byte aligned stages");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
@@ -624,17 +629,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     {
       const uint4* qc = reinterpret_cast<const uint4*>(a.q_c + qrow * kDc + crank * kHalfC);
       const uint4* qr = reinterpret_cast<const uint4*>(a.q_r + qrow * kDr + crank * kHalfR);
+      // both blocks' loads are issued before the first TMEM store (a single
+      // round trip to memory: the stores are barriers to the compiler)
+      uint32_t v[2][32];
 #pragma unroll
-      for (int bb = 0; bb < 2; ++bb) {
-        const int blk = 2 * h + bb;
-        uint32_t v[32];
+      for (int bb = 0; bb < 2; ++bb)
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint4 x = row_ok ? __ldg(qc + blk * 8 + k) : make_uint4(0, 0, 0, 0);
-          v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+          const uint4 x = row_ok ? __ldg(qc + (2 * h + bb) * 8 + k) : make_uint4(0, 0, 0, 0);
+          v[bb][4 * k] = x.x; v[bb][4 * k + 1] = x.y; v[bb][4 * k + 2] = x.z; v[bb][4 * k + 3] = x.w;
         }
-        ptx::tmem_st32(lane_base + kTmemQ + blk * 32, v);
-      }
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb) ptx::tmem_st32(lane_base + kTmemQ + (2 * h + bb) * 32, v[bb]);
       uint8_t* qrs = smem + kOffQR + (i >> 3) * 512 + (i & 7) * 16;
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
@@ -875,15 +881,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
       const float lse = l_tot > 0.0f ? (m_used + log2f(l_tot)) * kLn2 : -CUDART_INF_F;
       const size_t part = (static_cast<size_t>(b) * a.n_split + split) * a.rows + row;
+      // My 128 channels of the row are staged in shared memory, then written
+      // by one bulk copy: whole 128-byte lines, where direct stores would
+      // scatter 16-byte pieces over 32 rows per warp instruction.
+      const bool bf16_out = (a.n_split == 1 && !a.out_f32);
+      uint8_t* srow = smem + kOffC + i * kEpiRow + h * 512;
 #pragma unroll 1
       for (int c = 0; c < kHalfC / 64; ++c) {
         uint32_t ov[32];
         ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
         ptx::tmem_ld_wait();
-        const int col = crank * kHalfC + h * (kHalfC / 2) + c * 32;
-        if (!row_ok) continue;
-        if (a.n_split == 1 && !a.out_f32) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc + col);
+        if (bf16_out) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             uint32_t w[4];
@@ -893,17 +901,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                         __uint_as_float(ov[8 * k + 2 * e + 1]) * inv);
               w[e] = *reinterpret_cast<uint32_t*>(&hv);
             }
-            dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(srow + c * 64 + 16 * k) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          float* base = (a.n_split == 1) ? static_cast<float*>(a.out) + qrow * kDc + col
-                                         : a.o_part + part * kDc + col;
-          float4* dst = reinterpret_cast<float4*>(base);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
-                                 __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
+            *reinterpret_cast<float4*>(srow + c * 128 + 16 * k) =
+                make_float4(__uint_as_float(ov[4 * k]) * inv, __uint_as_float(ov[4 * k + 1]) * inv,
+                            __uint_as_float(ov[4 * k + 2]) * inv, __uint_as_float(ov[4 * k + 3]) * inv);
         }
+      }
+      if (row_ok) {
+        const int col = crank * kHalfC + h * (kHalfC / 2);
+        void* dst = bf16_out ? static_cast<void*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc + col)
+                             : static_cast<void*>((a.n_split == 1 ? static_cast<float*>(a.out) + qrow * kDc
+                                                                  : a.o_part + part * kDc) + col);
+        ptx::fence_proxy_async_smem();
+        ptx::bulk_store(dst, srow, bf16_out ? 256u : 512u);
+        ptx::bulk_commit();
+        ptx::bulk_wait_all();  // the copy has read shared memory and written the row before the CTA exits
       }
       if (crank == 0 && h == 0 && row_ok) {
         if (a.n_split == 1) {
