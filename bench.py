@@ -496,6 +496,42 @@ def main():
                       "cache_bytes": q_bytes + b_bytes,
                       "compression_vs_bf16": int(lens.astype(np.int64).sum()) * 1152 / (q_bytes + b_bytes)}
 
+    # ---- the same step replayed from a CUDA graph (one graph launch per R steps) ----
+    graph_leg = None
+    try:
+        def step_cur(k):  # launches on the current stream (the capture stream while capturing)
+            api.mla_qdecode_fused_append(desc, pools[k], table_t, lens_t, max_len, newc_t, newr_t, qcs[k], qrs[k],
+                                         w.scale, out=out, lse=lse, num_splits=w.num_splits, workspace=ws)
+        cs = torch.cuda.Stream(device=dev)
+        cs.wait_stream(stream)
+        with torch.cuda.stream(cs):
+            for k in range(R):
+                step_cur(k)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cs, capture_error_mode="relaxed"):
+            for k in range(R):
+                step_cur(k)
+        torch.cuda.synchronize()
+        reps = max(1, args.steps // R)
+        for _ in range(max(1, args.warmup // R)):
+            graph.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(reps):
+            graph.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        ms_g = g0.elapsed_time(g1) / (reps * R)
+        assert api.mla_get_device_status() == 0
+        graph_leg = {"ms_per_step": ms_g, "head_tokens_per_s": job_rate(st["head_tokens"], 1, ms_g),
+                     "steps_per_replay": R, "replays": reps}
+        del graph
+    except Exception as exc:  # capture unsupported here: report it, keep the other legs
+        torch.cuda.synchronize()
+        graph_leg = {"unavailable": f"{type(exc).__name__}: {exc}"[:200]}
+
     # ---- end to end through the C ABI with host buffers ----
     h_qc = torch.from_numpy(qc_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     h_qr = torch.from_numpy(qr_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -578,6 +614,7 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "bf16_decode": bf16_leg,
         "hybrid_decode": hybrid_leg,
+        "cuda_graph": graph_leg,
         "clocks": clk.summary(),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
