@@ -35,10 +35,17 @@
 //   warps 2-5   unpack + dequantize into bf16 hi/lo operand tiles
 //   warps 8-15  two threads per row (warps w and w+4 share a TMEM lane
 //               quarter, 16 of each chunk's 32 columns each): score exchange,
-//               online softmax, P tiles,
-//               output rescaling in TMEM, epilogue
+//               online softmax, P tiles, output rescaling in TMEM, epilogue
+//               (rows staged in shared memory and written by bulk copies)
+// Fused append (mla_qdecode_fused_append): before the cluster barrier of the
+// set-up, CTA 0's softmax warps quantize the step's new tokens that fall in
+// the unit's key range into the pool; the barrier and proxy fences order
+// those writes before both CTAs' TMA reads.
+// The host caps a unit at 8,192 keys: the fp32 accumulation in TMEM loses
+// accuracy in proportion to the keys one accumulator sums.
 // Every wait is bounded; a timeout sets MLA_ERR_TIMEOUT and the unit drains
-// and exits without touching memory it does not own.
+// and exits without touching memory it does not own. The kernel is launched
+// as a programmatic dependent and waits (griddepcontrol.wait) before any read.
 #include <cuda.h>
 #include <math_constants.h>
 
