@@ -73,6 +73,15 @@ def test_split_plan_and_workspace(lib):
     assert lib.mla_decode_workspace_bytes(1, 1, 16, 64, 1) == 0
     n = lib.mla_decode_num_splits(32, 1, 128, 4096, 0)
     assert 1 <= n <= 64
+    # no chunk sums more than 8,192 keys: explicit requests are raised, automatic plans respect it
+    assert lib.mla_decode_num_splits(1, 1, 128, 8192, 1) == 1
+    assert lib.mla_decode_num_splits(1, 1, 128, 8193, 1) == 2
+    assert lib.mla_decode_num_splits(1, 1, 128, 32768, 1) == 4
+    assert lib.mla_decode_num_splits(1, 1, 128, 32768, 8) == 8
+    for B, T in ((1, 1 << 20), (128, 32768), (4, 131072), (64, 16384)):
+        n = lib.mla_decode_num_splits(B, 1, 128, T, 0)
+        pages = (T + 63) // 64
+        assert (pages + n - 1) // n <= 128, (B, T, n)
 
 
 FAKE = 0x10000000  # never dereferenced: every call below fails validation first
