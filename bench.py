@@ -358,15 +358,11 @@ def main():
     torch.cuda.synchronize()
     assert api.mla_get_device_status() == 0
 
-    def step(k, ev=None):
+    def step(k):
         # the step's append of its new tokens and the decode, in one C-ABI call
         # (the append runs inside the decode kernel where the tensor-core path applies)
-        if ev is not None:
-            ev[0].record(stream)
         api.mla_qdecode_fused_append(desc, pools[k], table_t, lens_t, max_len, newc_t, newr_t, qcs[k], qrs[k],
                                      w.scale, out=out, lse=lse, num_splits=w.num_splits, workspace=ws, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
 
     def step_separate(k, ev):
         # the same step as two calls: mla_qcache_append, then mla_qdecode
