@@ -98,6 +98,16 @@ def workload_stats(w, lens):
                 alg_bytes_bf16=alg_bytes_bf16, flops=flops, q_bytes=q_bytes, o_bytes=o_bytes)
 
 
+def append_stats(w, ms):
+    """Rate of the cache append of one step (B * n_new tokens) taking ms milliseconds: tokens/s and
+    GB/s over its algorithmic bytes (bf16 tokens read, packed codes and metadata written)."""
+    tokens = w.B * w.n_new
+    bpt = (512 * w.bits_c // 8 + (512 // w.group_c) * 4 + 64 * w.bits_r // 8 + (64 // w.group_r) * 4)
+    nbytes = tokens * (576 * 2 + bpt)
+    return {"tokens": tokens, "ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "bytes": nbytes}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples over a region."""
 
@@ -605,6 +615,7 @@ def main():
                 "note": "algorithmic bytes of one decode / decode-call time"},
         "legs_ms": {"fused_append_decode": ms_decode,
                     "separate": {"append": ms_append, "decode": ms_sep_decode, "sum": ms_append + ms_sep_decode}},
+        "append": append_stats(w, ms_append),
         "roofline": roof,
         "e2e": {"value": job_rate(st["head_tokens"], world, ms_e2e), "unit": "head-tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},

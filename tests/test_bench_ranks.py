@@ -63,3 +63,13 @@ def test_reference_arm_other_ranks_exit_without_work():
                        timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_append_stats_closed_form():
+    # 32 requests x 1 token of INT4/INT4 g64: 1152 B read + 324 B written per token
+    from bit_mla_kv_qdecode_b200 import synth
+    a = bench.append_stats(synth.workload("dsv3"), 0.01)
+    assert a["tokens"] == 32 and a["bytes"] == 32 * (1152 + 324)
+    assert abs(a["tokens_per_s"] - 3.2e6) < 1e-3 and abs(a["gbs"] - 32 * 1476 / 1e-5 / 1e9) < 1e-9
+    m = bench.append_stats(synth.workload("mtp"), 0.02)  # INT2 g32 content: 228 B per token, 2 tokens each
+    assert m["tokens"] == 256 and m["bytes"] == 256 * (1152 + 228)
