@@ -422,6 +422,7 @@ mla_status mla_qdecode_hybrid(const mla_qcache_desc* desc, const void* pool, con
   if (B < 0 || s_q < 1 || H < 1 || max_hist_len < 0 || max_prot_len < 0) return MLA_ERR_INVALID_ARG;
   if (out_dtype != 0 && out_dtype != 1) return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
+  if (static_cast<long>(B) * s_q * H > 0x7FFFFFFFL) return MLA_ERR_UNSUPPORTED;  // rows of the merge
   if (!out || !q_c || !q_r || !aligned(out, 16) || !aligned(lse, 4)) return MLA_ERR_INVALID_ARG;
   const HybridWorkspace hw = hybrid_workspace(B, s_q, H, max_hist_len, max_prot_len);
   if (!workspace || workspace_bytes < hw.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;

@@ -174,3 +174,33 @@ def test_fused_append_argument_errors(lib):
     assert call(pool=None) == E.MLA_ERR_INVALID_ARG
     assert call(B=0) == E.MLA_OK
     assert call(B=0, n=0, cn=None, kn=None) == E.MLA_OK
+
+
+def test_hybrid_and_noalloc_argument_errors(lib):
+    E = _lib
+    d = ctypes.byref(_lib.make_desc(4, 64, num_pages=8))
+
+    def hybrid(B=2, s_q=1, H=16, out=FAKE, ws=FAKE, ws_bytes=1 << 30, out_dtype=0, desc=d):
+        return lib.mla_qdecode_hybrid(desc, FAKE, FAKE, 4, FAKE, 128, FAKE, 4, FAKE, 4, FAKE, 128, FAKE, FAKE,
+                                      B, s_q, H, 0.1, ws, ws_bytes, out, out_dtype, None, None)
+
+    assert hybrid(B=0) == E.MLA_OK
+    assert hybrid(s_q=0) == E.MLA_ERR_INVALID_ARG
+    assert hybrid(out_dtype=3) == E.MLA_ERR_INVALID_ARG
+    assert hybrid(out=None) == E.MLA_ERR_INVALID_ARG
+    assert hybrid(ws=None) == E.MLA_ERR_WORKSPACE
+    assert hybrid(ws_bytes=16) == E.MLA_ERR_WORKSPACE
+    assert hybrid(B=60000, s_q=4, H=16384) == E.MLA_ERR_UNSUPPORTED
+    assert hybrid(desc=ctypes.byref(_lib.make_desc(3, 64))) == E.MLA_ERR_UNSUPPORTED
+    # page moves: B == 0 is a no-op; missing pointers are argument errors
+    assert lib.mla_qcache_append_bf16_pages(d, FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, 0, None) == E.MLA_OK
+    assert lib.mla_qcache_append_bf16_pages(d, FAKE, FAKE, 4, FAKE, FAKE, 4, None, 2, None) == E.MLA_ERR_INVALID_ARG
+    # allocation-free decode: its argument errors come before any device work
+    assert lib.mla_qdecode_noalloc(d, FAKE, FAKE, 4, FAKE, 256, FAKE, FAKE, -1, 1, 16, 0.1, 0, FAKE, 0, None, 0,
+                                   None) == E.MLA_ERR_INVALID_ARG
+    assert lib.mla_qdecode_noalloc(d, FAKE, FAKE, 4, FAKE, 256, FAKE, FAKE, 2, 0, 16, 0.1, 0, FAKE, 0, None, 0,
+                                   None) == E.MLA_ERR_INVALID_ARG
+    # a plan whose split scratch exceeds the fixed array is refused, not truncated
+    big = lib.mla_qdecode_noalloc(d, FAKE, FAKE, 4096, FAKE, 262144, FAKE, FAKE, 64, 1, 128, 0.1, 32, FAKE, 0, None,
+                                  0, None)
+    assert big == E.MLA_ERR_WORKSPACE
