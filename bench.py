@@ -5,7 +5,7 @@ the step's new tokens (mla_qcache_append), then the decode over the quantized
 cache (mla_qdecode: split-KV decode kernel + combine). The BF16 comparison
 decode (mla_decode_bf16) is timed as a separate leg on the same shapes.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dsv3]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mtp]
   python bench.py --impl reference ...    # the CPU oracle, timed on host cores
 
 Prints one JSON line on rank 0. Inputs are synthetic (seeded; see
@@ -284,7 +284,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="dsv3")
+    # default: the largest workload that fits one GPU (B=128, H=128, s_q=2 causal,
+    # ragged T in [1024, 32768], INT2/INT4, 2 tokens appended per request and step)
+    ap.add_argument("--workload", default="mtp")
     ap.add_argument("--batch", type=int, default=0,
                     help="run the workload with this many requests instead (small cases for profiling)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -426,12 +428,15 @@ def main():
     peaks, peak_src = load_peaks()
     flop_rate = st["flops"] / (ms_decode * 1e-3) / 1e12
     gbs = st["alg_bytes"] / (ms_decode * 1e-3) / 1e9
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    # The timed region lasts well under the seconds-long loop behind the sustained
+    # figure, so the burst bf16 peak is the denominator.
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     tensor_bound = st["flops"] / st["alg_bytes"] > ridge
     if tensor_bound:
-        roof = {"bound": "tensor", "achieved": flop_rate, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": flop_rate / peaks["bf16_tflops_sustained"], "traffic": None,
-                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+        roof = {"bound": "tensor", "achieved": flop_rate, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": flop_rate / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops (burst: the timed region is "
+                               f"{ms_total:.0f} ms, not a seconds-long loop)"}
     else:
         roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peak_src} hbm_gbs"}

@@ -358,11 +358,13 @@ mla_status mla_bf16cache_append(void* pool, int num_pages, int page_size, const 
 
 int mla_decode_num_splits(int B, int s_q, int H, int max_seq_len, int num_splits) {
   if (B < 0 || s_q < 1 || H < 1 || max_seq_len < 0 || num_splits < 0) return 0;
+  if (static_cast<long>(s_q) * H > (1 << 20)) return 0;  // beyond what a decode accepts; s_q * H must not overflow
   return plan_splits(B, s_q, H, max_seq_len, num_splits).n_split;
 }
 
 size_t mla_decode_workspace_bytes(int B, int s_q, int H, int max_seq_len, int num_splits) {
   if (B <= 0 || s_q < 1 || H < 1 || max_seq_len < 0 || num_splits < 0) return 0;
+  if (static_cast<long>(s_q) * H > (1 << 20)) return 0;  // beyond what a decode accepts; s_q * H must not overflow
   return workspace_for(B, s_q * H, plan_splits(B, s_q, H, max_seq_len, num_splits));
 }
 

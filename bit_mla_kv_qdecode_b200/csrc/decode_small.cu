@@ -163,7 +163,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
       ptx::mbar_arrive_expect_tx(&full[s], G::kPageBytes);
       ptx::bulk_load(smem + s * Lo::kStage, a.pool + static_cast<size_t>(page) * G::kPageBytes, G::kPageBytes,
                      &full[s]);
-    } else {
+    } else {  // never dereferenced: the page's keys are masked and the call is flagged
+      record_error(a.status, MLA_ERR_INVALID_ARG);
       stage_page[s] = -1;
       ptx::mbar_arrive(&full[s]);
     }

@@ -162,11 +162,13 @@ mla_status mla_bf16cache_append(void* pool, int num_pages, int page_size,
 /* Number of key splits the decode calls use for this shape: num_splits if it
  * is > 0 (capped at the page count of max_seq_len), otherwise the library's
  * choice for the current device. 1 means no split and no workspace. Host only
- * (queries the current device's SM count; assumes 148 SMs without a GPU). */
+ * (queries the current device's SM count; assumes 148 SMs without a GPU).
+ * Returns 0 for arguments no decode accepts (negative sizes, s_q * H > 2^20). */
 int mla_decode_num_splits(int B, int s_q, int H, int max_seq_len, int num_splits);
 
 /* Workspace bytes mla_qdecode / mla_decode_bf16 need for this shape and
- * split request (0 when the plan has a single split). Host only. */
+ * split request (0 when the plan has a single split, and for arguments no
+ * decode accepts: B <= 0, negative sizes, s_q * H > 2^20). Host only. */
 size_t mla_decode_workspace_bytes(int B, int s_q, int H, int max_seq_len, int num_splits);
 
 /* Low-bit MLA decode in the absorbed MQA form over a quantized paged cache.

@@ -89,28 +89,67 @@ def oracle_request(case: Case, b: int, quantized=True):
     return C, R
 
 
-def oracle_decode(case: Case, requests, quantized=True):
-    """{b: (o [s_q, H, 512], lse [s_q, H])} for the listed requests."""
+def _oracle_rows(case: Case, b: int, C, R, heads=None):
+    """Oracle (o [s_q, H', 512], lse [s_q, H']) of request b over its dequantized keys,
+    for every head or only the listed ones."""
     w = case.w
-    res = {}
-    qc = synth.bf16_bits_to_f32(case.qc_bits)
-    qr = synth.bf16_bits_to_f32(case.qr_bits)
-    for b in requests:
-        C, R = oracle_request(case, b, quantized)
-        rq_c, rq_r, L = attention.request_rows(qc[b], qr[b], int(case.lens[b]))
-        o, lse = attention.attend(rq_c, rq_r, C, R, w.scale, L)
-        res[b] = (o.reshape(w.s_q, w.H, -1), lse.reshape(w.s_q, w.H))
-    return res
+    qc = synth.bf16_bits_to_f32(case.qc_bits[b])
+    qr = synth.bf16_bits_to_f32(case.qr_bits[b])
+    if heads is not None:
+        qc, qr = qc[:, heads], qr[:, heads]
+    nh = qc.shape[1]
+    rq_c, rq_r, L = attention.request_rows(qc, qr, int(case.lens[b]))
+    o, lse = attention.attend(rq_c, rq_r, C, R, w.scale, L)
+    return o.reshape(w.s_q, nh, -1), lse.reshape(w.s_q, nh)
+
+
+def oracle_decode(case: Case, requests, quantized=True, heads=None):
+    """{b: (o [s_q, H', 512], lse [s_q, H'])} for the listed requests (H' = len(heads))."""
+    return {b: _oracle_rows(case, b, *oracle_request(case, b, quantized), heads=heads) for b in requests}
+
+
+def fill_pool_with_reference(case: Case, heads, upto="all", chunk=8192, all_heads=()):
+    """fill_pool and oracle_decode(heads=...) over every request in one pass: each
+    request's tokens are drawn once, appended through the library (its first n
+    tokens, n = lens or n_history) and quantized by the oracle (all lens tokens).
+    Returns (pool, table, ref over `heads` for every request, ref over every head
+    for the requests listed in all_heads)."""
+    dev = "cuda"
+    w = case.w
+    table_t = torch.from_numpy(case.table).to(dev)
+    pool = api.new_qcache_pool(case.desc)
+    ref, ref_all = {}, {}
+    for b in range(w.B):
+        toks = case.tokens(b)
+        n = int(case.lens[b] if upto == "all" else case.n_history[b])
+        for t0 in range(0, n, chunk):
+            part = toks[t0:min(t0 + chunk, n)]
+            lb = torch.tensor([t0], dtype=torch.int32, device=dev)
+            api.mla_qcache_append(case.desc, pool, table_t[b:b + 1], lb, bits_to_torch(part[None, :, :512]),
+                                  bits_to_torch(part[None, :, 512:]))
+        x = synth.bf16_bits_to_f32(toks)
+        u, s, z = quant.quantize_groups(x[:, :512], w.bits_c, w.group_c)
+        C = quant.dequantize_groups(u, s, z, w.group_c)
+        u, s, z = quant.quantize_groups(x[:, 512:], w.bits_r, w.group_r)
+        R = quant.dequantize_groups(u, s, z, w.group_r)
+        ref[b] = _oracle_rows(case, b, C, R, heads=heads)
+        if b in all_heads:
+            ref_all[b] = _oracle_rows(case, b, C, R)
+    return pool, table_t, ref, ref_all
 
 
 def device_queries(case: Case):
     return bits_to_torch(case.qc_bits), bits_to_torch(case.qr_bits)
 
 
-def parity(out: torch.Tensor, lse: torch.Tensor, ref: dict, bf16_out=False):
-    """Return (err / RMS, max |lse diff|) over the requests in ref; assert nothing."""
+def parity(out: torch.Tensor, lse: torch.Tensor, ref: dict, bf16_out=False, heads=None):
+    """Return (err / RMS, max |lse diff|) over the requests in ref (and, when given,
+    only the listed heads, as oracle_decode(heads=...) computed them); assert nothing."""
     o_dev = out.float().cpu().numpy()
     l_dev = lse.cpu().numpy() if lse is not None else None
+    if heads is not None:
+        o_dev = o_dev[:, :, heads]
+        l_dev = l_dev[:, :, heads] if l_dev is not None else None
     refs = np.concatenate([ref[b][0].reshape(-1) for b in ref])
     rms = float(np.sqrt(np.mean(refs ** 2))) if refs.size else 1.0
     worst, lworst = 0.0, 0.0

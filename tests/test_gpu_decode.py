@@ -135,8 +135,28 @@ def test_split_counts_agree():
 
 
 # Full-size workloads in the launch configuration the benchmark times (auto
-# split plan, bf16 output), oracle on a sample of requests.
-FULL = {0: [0], 1: [0, 31], 2: [5, 40], 3: [2], 4: [0, 77], 5: [3]}
+# split plan, bf16 output), oracle on a sample of requests. The ragged
+# workloads (2 and 4) are checked on every request below.
+FULL = {0: [0], 1: [0, 31], 3: [2], 5: [3]}
+
+# A fixed subset of heads for the every-request checks: the oracle's cost grows
+# with the heads it evaluates, while the kernels treat every head alike (the
+# first and last rows of each 128-row tile are among them).
+HEADS = [0, 45, 90, 127]
+
+
+@pytest.mark.parametrize("idx", [2, 4])
+def test_full_size_every_request(idx):
+    w = synth.workload(idx)
+    case = mc.make_case(w)
+    pool, table_t, ref, ref_all = mc.fill_pool_with_reference(case, HEADS, all_heads=(5, w.B - 1))
+    out, lse = run_decode(case, pool, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16)
+    assert api.mla_get_device_status() == 0
+    assert len(ref) == w.B
+    err, lerr = mc.parity(out, lse, ref, bf16_out=True, heads=HEADS)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
+    err, lerr = mc.parity(out, lse, ref_all, bf16_out=True)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
 
 
 @pytest.mark.parametrize("idx", sorted(FULL))

@@ -80,3 +80,33 @@ def test_fused_length_below_n_new_is_flagged():
     torch.cuda.synchronize()
     assert api.mla_get_device_status() == api._lib.MLA_ERR_INVALID_ARG
     assert api.mla_get_device_status() == 0  # reading clears it
+
+
+def test_fused_full_size_mtp_every_request():
+    """The benchmark's timed call on the full speculative-verify workload (128
+    requests, 128 heads, 2 causal queries, ragged 1K..32K keys, INT2/INT4, 2 new
+    tokens per request): auto split plan, bf16 output, checked against the oracle
+    on every request (a fixed head subset) and on two requests in full. The plain
+    decode over the pool the fused call left must then give the same bits."""
+    heads = [0, 45, 90, 127]
+    w = synth.workload(4)
+    case = mc.make_case(w)
+    pool, table_t, ref, ref_all = mc.fill_pool_with_reference(case, heads, upto="history", all_heads=(0, 77))
+    c_new, kr_new = _new_tokens(case)
+    qc, qr = mc.device_queries(case)
+    lens_t = torch.from_numpy(case.lens).cuda()
+    lse = torch.empty((w.B, w.s_q, w.H), dtype=torch.float32, device="cuda")
+    out, _ = api.mla_qdecode_fused_append(case.desc, pool, table_t, lens_t, case.max_seq_len, c_new, kr_new,
+                                          qc, qr, w.scale, out_dtype=torch.bfloat16, lse=lse,
+                                          num_splits=w.num_splits)
+    torch.cuda.synchronize()
+    assert api.mla_get_device_status() == 0
+    err, lerr = mc.parity(out, lse, ref, bf16_out=True, heads=heads)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
+    err, lerr = mc.parity(out, lse, ref_all, bf16_out=True)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
+    lse2 = torch.empty_like(lse)
+    out2, _ = api.mla_qdecode(case.desc, pool, table_t, lens_t, case.max_seq_len, qc, qr, w.scale,
+                              out_dtype=torch.bfloat16, lse=lse2, num_splits=w.num_splits)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
