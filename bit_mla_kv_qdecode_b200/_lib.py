@@ -25,6 +25,7 @@ MLA_ERR_TIMEOUT = 6
 MLA_DECODE_DEFAULT = 0
 MLA_DECODE_FORCE_SIMT = 1
 MLA_DECODE_FAST_UNCOMPENSATED = 2
+MLA_DECODE_TEST_STALL = 4  # tests only: runs the device-side timeout path
 
 MLA_QDECODE_NOALLOC_SCRATCH_BYTES = 64 << 20
 

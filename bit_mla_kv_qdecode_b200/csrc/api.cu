@@ -154,7 +154,8 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
     return MLA_ERR_INVALID_ARG;
   if (c.out_dtype != 0 && c.out_dtype != 1) return MLA_ERR_INVALID_ARG;
   if (!isfinite(c.scale)) return MLA_ERR_INVALID_ARG;
-  if (c.flags & ~(MLA_DECODE_FORCE_SIMT | MLA_DECODE_FAST_UNCOMPENSATED)) return MLA_ERR_INVALID_ARG;
+  if (c.flags & ~(MLA_DECODE_FORCE_SIMT | MLA_DECODE_FAST_UNCOMPENSATED | MLA_DECODE_TEST_STALL))
+    return MLA_ERR_INVALID_ARG;
   if (c.n_new < 0 || (c.n_new > 0 && (!quantized || !c.c_new || !c.kr_new))) return MLA_ERR_INVALID_ARG;
   if (c.n_new > 0 && (!aligned(c.c_new, 16) || !aligned(c.kr_new, 16) || !c.pool)) return MLA_ERR_INVALID_ARG;
   if (static_cast<long>(c.B) * c.n_new > (1L << 26)) return MLA_ERR_UNSUPPORTED;

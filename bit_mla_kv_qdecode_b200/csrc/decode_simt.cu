@@ -338,6 +338,7 @@ DecodeArgs make_decode_args(const DecodeLaunch& L) {
   a.c_new = static_cast<const __nv_bfloat16*>(L.c_new);
   a.kr_new = static_cast<const __nv_bfloat16*>(L.kr_new);
   a.n_new = L.n_new;
+  a.flags = L.flags;
   return a;
 }
 

@@ -68,6 +68,7 @@ constexpr int kHalfR = 32;            // rope channels per CTA
 constexpr int kKChunks = (kHalfC + kHalfR) / 8;  // 36 eight-channel chunks per token
 constexpr int kNC = 3;                // operand-tile stages
 constexpr int kNS = 4;                // TMA code stages
+static_assert(kChunk == 32, "the PV issue sequence covers two 16-token K-steps");
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (weights stay <= 2^8)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr unsigned kFull = 0xffffffffu;
@@ -272,6 +273,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t crank = ptx::cluster_ctarank();
   const uint32_t peer = crank ^ 1u;
+  // MLA_DECODE_TEST_STALL (tests only): every wait gives up after 1 ms and the
+  // page producer never issues chunk 1, so that the timeout path runs
+  const bool test_stall = (a.flags & MLA_DECODE_TEST_STALL) != 0;
+  const uint64_t wlim = test_stall ? 1000000ull : kWaitLimitNs;
 
   // ---- unit ----
   const int unit = blockIdx.x >> 1;
@@ -388,10 +393,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kNC; ++i) issued[i] = 0;
       for (int j = 0; j < n_chunks; ++j) {
         const int cs = j % kNC;
-        if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, kWaitLimitNs)) {
+        if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, wlim)) {
           fail(a, abort_flag);
           break;
         }
+        if (test_stall && j == 1) continue;  // never issued nor arrived: the consumers' waits run out
         const int t0 = t_begin + j * kChunk;
         const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
         uint8_t* st = smem + kOffC + cs * kCStage;
@@ -409,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         issued[cs] = j + 1;
       }
       for (int cs = 0; cs < kNC; ++cs)
-        if (issued[cs] > 0) ptx::mbar_wait(&bars.code_full[cs], ((issued[cs] - 1) / kNC) & 1, nullptr, kWaitLimitNs);
+        if (issued[cs] > 0) ptx::mbar_wait(&bars.code_full[cs], ((issued[cs] - 1) / kNC) & 1, nullptr, wlim);
     } else if (lane == 0) {
       if (a.n_new > 0) ptx::fence_proxy_async_global();  // the fused append's writes precede these TMA reads
       const uint32_t bytes = kChunk * (G::kRowC / 2) + kChunk * G::kRowR + kChunk * (G::kGroupsC * 2) +
@@ -418,10 +424,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kNS; ++i) issued[i] = 0;
       for (int j = 0; j < n_chunks; ++j) {
         const int s = j % kNS;
-        if (j >= kNS && !ptx::mbar_wait(&bars.code_empty[s], ((j - kNS) / kNS) & 1, abort_flag, kWaitLimitNs)) {
+        if (j >= kNS && !ptx::mbar_wait(&bars.code_empty[s], ((j - kNS) / kNS) & 1, abort_flag, wlim)) {
           fail(a, abort_flag);
           break;
         }
+        if (test_stall && j == 1) continue;  // never issued nor arrived: the consumers' waits run out
         const int t0 = t_begin + j * kChunk;
         const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
         uint8_t* st = smem + kOffCode + s * kCodeStage;
@@ -444,7 +451,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       // drain copies still in flight before the CTA can exit
       for (int s = 0; s < kNS; ++s)
-        if (issued[s] > 0) ptx::mbar_wait(&bars.code_full[s], ((issued[s] - 1) / kNS) & 1, nullptr, kWaitLimitNs);
+        if (issued[s] > 0) ptx::mbar_wait(&bars.code_full[s], ((issued[s] - 1) / kNS) & 1, nullptr, wlim);
     }
   } else if (warp == 1 || warp == 7) {
     // =========================== QK issuers ===========================
@@ -461,11 +468,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t idesc = ptx::idesc_bf16_f32(kRows, (!kBF16 && n_terms_qk == 2) ? 2 * kChunk : kChunk, 0, 0);
       const uint64_t b0 = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffC), cstride, 128);
       const uint64_t a_rope = ptx::smem_desc_noswizzle(ptx::smem_u32(smem + kOffQR), 128, 512);
-      bool ok = ptx::mbar_wait(bars.q_full, 0, abort_flag, kWaitLimitNs);
+      bool ok = ptx::mbar_wait(bars.q_full, 0, abort_flag, wlim);
       for (int j = par; ok && j < n_chunks; j += 2) {
         const int cs = j % kNC, sb = j & 1;
-        if (!ptx::mbar_wait(&bars.c_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs) ||
-            (j >= 2 && !ptx::mbar_wait(&bars.s_empty[sb], ((j - 2) >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!ptx::mbar_wait(&bars.c_full[cs], (j / kNC) & 1, abort_flag, wlim) ||
+            (j >= 2 && !ptx::mbar_wait(&bars.s_empty[sb], ((j - 2) >> 1) & 1, abort_flag, wlim))) {
           ok = false;
           break;
         }
@@ -477,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < kHalfC / 16; ++k) {
           if (k == kHalfC / 32) {
-            if (!ptx::mbar_wait(&bars.c_full2[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) {
+            if (!ptx::mbar_wait(&bars.c_full2[cs], (j / kNC) & 1, abort_flag, wlim)) {
               ok = false;
               break;
             }
@@ -495,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) fail(a, abort_flag);
       ptx::mma_commit(drain);
-      ptx::mbar_wait(drain, 0, nullptr, kWaitLimitNs);  // MMAs finish before TMEM is released
+      ptx::mbar_wait(drain, 0, nullptr, wlim);  // MMAs finish before TMEM is released
     }
   } else if (warp == 6) {
     // =========================== PV issuer ===========================
@@ -508,27 +515,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int j = 0; j < n_chunks; ++j) {
         const int pb = j & 1, cs = j % kNC;
-        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, wlim)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
+        // Straight-line issue: the issuing thread runs no per-instruction
+        // address or predicate arithmetic between the MMAs (measured: such
+        // work between two tcgen05.mma instructions slows their issue).
         const uint64_t ap = a0 + static_cast<uint64_t>((pb * 2 * kPTile) >> 4);
         const uint64_t bc = b0 + static_cast<uint64_t>((cs * kCStage) >> 4);
-        for (int term = 0; term < n_terms_pv; ++term) {
-          const uint64_t at = ap + (term == 1 ? static_cast<uint64_t>(kPTile >> 4) : 0);   // P_lo for term 1
-          const uint64_t bt = bc + (term == 2 ? static_cast<uint64_t>(kCLoOff >> 4) : 0);  // C_lo for term 2
-#pragma unroll
-          for (int k = 0; k < kChunk / 16; ++k)
-            ptx::mma_ss(tmem + kTmemO, at + static_cast<uint64_t>((k * 256) >> 4),
-                        bt + static_cast<uint64_t>((k * 256) >> 4), idesc, (j > 0 || term > 0 || k > 0) ? 1u : 0u);
+        const uint64_t ap_lo = ap + static_cast<uint64_t>(kPTile >> 4);    // P_lo
+        const uint64_t bc_lo = bc + static_cast<uint64_t>(kCLoOff >> 4);   // C_lo
+        constexpr uint64_t kK1 = 256 >> 4;                                 // second 16-token K-step
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+        const uint32_t o = tmem + kTmemO;
+        ptx::mma_ss(o, ap, bc, idesc, acc0);                               // P_hi . C_hi
+        ptx::mma_ss(o, ap + kK1, bc + kK1, idesc, 1u);
+        if (n_terms_pv >= 2) {                                             // P_lo . C_hi
+          ptx::mma_ss(o, ap_lo, bc, idesc, 1u);
+          ptx::mma_ss(o, ap_lo + kK1, bc + kK1, idesc, 1u);
+        }
+        if (n_terms_pv >= 3) {                                             // P_hi . C_lo
+          ptx::mma_ss(o, ap, bc_lo, idesc, 1u);
+          ptx::mma_ss(o, ap + kK1, bc_lo + kK1, idesc, 1u);
         }
         ptx::mma_commit(&bars.p_empty[pb]);
         ptx::mma_commit(&bars.c_empty[cs]);
       }
       if (!ok) fail(a, abort_flag);
       ptx::mma_commit(bars.o_full);
-      ptx::mbar_wait(bars.o_full, 0, nullptr, kWaitLimitNs);  // MMAs finish before TMEM is released
+      ptx::mbar_wait(bars.o_full, 0, nullptr, wlim);  // MMAs finish before TMEM is released
     }
   } else if (warp >= 2 && warp < 6) {
     // =========================== dequant ===========================
@@ -540,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // rows, or a page the table could not name) are zeroed so that 0 * x
       // never meets a NaN or Inf
       const int cs = j % kNC;
-      if (!ptx::mbar_wait(&bars.code_full[cs], (j / kNC) & 1, abort_flag, kWaitLimitNs)) { fail(a, abort_flag); break; }
+      if (!ptx::mbar_wait(&bars.code_full[cs], (j / kNC) & 1, abort_flag, wlim)) { fail(a, abort_flag); break; }
       const int t0 = t_begin + j * kChunk;
       const int lim = stage_page[cs] >= 0 ? t_end - t0 : 0;
       if (lim < kChunk && tq >= lim) {
@@ -555,8 +572,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; !kBF16 && j < n_chunks; ++j) {
       const int s = j % kNS, cs = j % kNC;
-      if (!ptx::mbar_wait(&bars.code_full[s], (j / kNS) & 1, abort_flag, kWaitLimitNs)) { fail(a, abort_flag); break; }
-      if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, kWaitLimitNs)) {
+      if (!ptx::mbar_wait(&bars.code_full[s], (j / kNS) & 1, abort_flag, wlim)) { fail(a, abort_flag); break; }
+      if (j >= kNC && !ptx::mbar_wait(&bars.c_empty[cs], ((j - kNC) / kNC) & 1, abort_flag, wlim)) {
         fail(a, abort_flag);
         break;
       }
@@ -681,7 +698,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto store_weights = [&](int jj, const uint32_t (&ph)[8], const uint32_t (&pl)[8]) -> bool {
       const int pb = jj & 1;
       if (jj >= 2 &&
-          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, kWaitLimitNs)))
+          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, wlim)))
         return false;
       uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
 #pragma unroll
@@ -702,7 +719,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // do not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
       if (__any_sync(kFull, rescale && o_live)) {
         if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
-                                              kWaitLimitNs)))
+                                              wlim)))
           return false;
         ptx::tc_fence_after();
         const float f = (rescale && o_live) ? alpha : 1.0f;
@@ -738,7 +755,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (j >= 1) {
         const int jj = j - 1, pb = jj & 1;
         const int t0 = t_begin + jj * kChunk;
-        if (!__all_sync(kFull, ptx::mbar_wait(&bars.x_full[pb], (jj >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.x_full[pb], (jj >> 1) & 1, abort_flag, wlim))) {
           ok = false;
           break;
         }
@@ -774,7 +791,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         red_max[(pb * 2 + h) * kRows + i] = mt[0];
         ptx::mbar_arrive(&bars.pair_max[quarter * 2 + pb]);
         if (!__all_sync(kFull, ptx::mbar_wait(&bars.pair_max[quarter * 2 + pb], (jj >> 1) & 1, abort_flag,
-                                              kWaitLimitNs))) {
+                                              wlim))) {
           ok = false;
           break;
         }
@@ -828,7 +845,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // block-table entry of chunk j, checked one step later: issued before the wait to hide the load
         cur_page = table_entry(a.table, a.max_pages, b, t_begin + j * kChunk);
         // wait results are made warp-uniform: the TMEM loads below are warp-collective
-        if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, kWaitLimitNs))) {
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, wlim))) {
           ok = false;
           break;
         }
@@ -879,8 +896,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (!ok) fail(a, abort_flag);
     red_sum[h * kRows + i] = l_sum;
     ptx::mbar_arrive(&bars.pair_sum[quarter]);
-    const bool sums_ready = ptx::mbar_wait(&bars.pair_sum[quarter], 0, abort_flag, kWaitLimitNs);
-    const bool o_ready = ptx::mbar_wait(bars.o_full, 0, abort_flag, kWaitLimitNs);
+    const bool sums_ready = ptx::mbar_wait(&bars.pair_sum[quarter], 0, abort_flag, wlim);
+    const bool o_ready = ptx::mbar_wait(bars.o_full, 0, abort_flag, wlim);
     const int aborted = *abort_flag;
     if (__all_sync(kFull, sums_ready && o_ready && ok && !aborted)) {  // warp-uniform: TMEM loads are collective
       ptx::tc_fence_after();

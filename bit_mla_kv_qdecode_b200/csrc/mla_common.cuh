@@ -88,6 +88,7 @@ struct DecodeArgs {
   const __nv_bfloat16* c_new;   // fused append: [B, n_new, 512] (tensor-core kernel only)
   const __nv_bfloat16* kr_new;  // [B, n_new, 64]
   int n_new;                    // 0: no fused append
+  unsigned flags;               // MLA_DECODE_* bits of the call
 };
 
 // Keys visible to flattened row r = i*H + h of a request holding T keys.

@@ -105,6 +105,13 @@ typedef struct {
  * per product instead of a hi/lo pair). Faster; its error exceeds the
  * library's stated bound on long, diffuse attention. Never the default. */
 #define MLA_DECODE_FAST_UNCOMPENSATED 2u
+/* Tests only. The tensor-core decode kernel (s_q * H > 16) never loads its
+ * second chunk of keys and every device-side wait gives up after 1 ms, so the
+ * call runs the timeout path: the kernel drains and exits, the call returns,
+ * mla_get_device_status then reports MLA_ERR_TIMEOUT, and out and lse are
+ * undefined. Later calls without the flag are unaffected. Other kernels
+ * ignore it. */
+#define MLA_DECODE_TEST_STALL 4u
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* mla_status_string(mla_status s);
