@@ -96,10 +96,32 @@ SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
   return SplitPlan{(pages + chunk - 1) / chunk, chunk};
 }
 
+// Units of the tensor-core kernel (request, split, 128-row tile).
+long tc_units(int B, int rows, const SplitPlan& p) {
+  return static_cast<long>(B) * p.n_split * ((rows + 127) / 128);
+}
+
+// Whether the tensor-core kernel takes its units from a device-built work
+// list, longest first: for split plans whose grid runs in more than two waves
+// of its 2-CTA cluster slots, where the order of the units decides the tail.
+bool use_worklist(int B, int rows, const SplitPlan& p) {
+  if (rows <= mla::kSmallRows || p.n_split <= 1 || p.chunk_pages > mla::kMaxWorklistChunkPages) return false;
+  const long units = tc_units(B, rows, p);
+  return units > 2L * (device_sm_count() / 2) && units <= (1L << 24);
+}
+
+// Bytes of the split partials (lse, then o), 256-byte aligned.
+size_t partials_bytes(int B, int rows, const SplitPlan& p) {
+  const size_t parts = static_cast<size_t>(B) * p.n_split * rows;
+  return align_up(parts * sizeof(float), 256) + align_up(parts * mla::kDc * sizeof(float), 256);
+}
+
+// Workspace of a decode: the split partials, then the work list (int32 per unit) when used.
 size_t workspace_for(int B, int rows, const SplitPlan& p) {
   if (p.n_split <= 1) return 0;
-  const size_t parts = static_cast<size_t>(B) * p.n_split * rows;
-  return align_up(parts * sizeof(float), 256) + parts * mla::kDc * sizeof(float);
+  size_t bytes = partials_bytes(B, rows, p);
+  if (use_worklist(B, rows, p)) bytes += static_cast<size_t>(tc_units(B, rows, p)) * sizeof(int);
+  return bytes;
 }
 
 mla_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA; }
@@ -205,6 +227,8 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
     const size_t parts = static_cast<size_t>(c.B) * plan.n_split * rows;
     L.lse_part = static_cast<float*>(c.workspace);
     L.o_part = reinterpret_cast<float*>(static_cast<char*>(c.workspace) + align_up(parts * sizeof(float), 256));
+    if (use_worklist(c.B, rows, plan))
+      L.worklist = reinterpret_cast<int*>(static_cast<char*>(c.workspace) + partials_bytes(c.B, rows, plan));
   }
   L.out = c.out;
   L.out_f32 = c.out_dtype;

@@ -339,6 +339,7 @@ DecodeArgs make_decode_args(const DecodeLaunch& L) {
   a.kr_new = static_cast<const __nv_bfloat16*>(L.kr_new);
   a.n_new = L.n_new;
   a.flags = L.flags;
+  a.worklist = L.worklist;
   return a;
 }
 

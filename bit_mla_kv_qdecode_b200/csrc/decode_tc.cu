@@ -278,8 +278,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool test_stall = (a.flags & MLA_DECODE_TEST_STALL) != 0;
   const uint64_t wlim = test_stall ? 1000000ull : kWaitLimitNs;
 
-  // ---- unit ----
-  const int unit = blockIdx.x >> 1;
+  // ---- unit: from the work list (longest first) when the plan has one ----
+  const int unit = a.worklist ? __ldg(a.worklist + (blockIdx.x >> 1)) : static_cast<int>(blockIdx.x >> 1);
   const int rt = unit % row_tiles;
   const int split = (unit / row_tiles) % a.n_split;
   const int b = unit / (row_tiles * a.n_split);
@@ -1048,6 +1048,10 @@ cudaError_t launch_t(const DecodeLaunch& L) {
   const int row_tiles = (a.rows + kRows - 1) / kRows;
   const long units = static_cast<long>(a.B) * a.n_split * row_tiles;
   if (units * 2 > 0x7FFFFFFFL) return cudaErrorNotSupported;
+  if (L.worklist) {
+    const cudaError_t pe = launch_plan_units(L, row_tiles);
+    if (pe != cudaSuccess) return pe;
+  }
   auto kern = decode_tc_kernel<BC, GC, BR, GR, kBF16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (e != cudaSuccess) return e;

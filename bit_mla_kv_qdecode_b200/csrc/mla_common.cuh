@@ -89,6 +89,7 @@ struct DecodeArgs {
   const __nv_bfloat16* kr_new;  // [B, n_new, 64]
   int n_new;                    // 0: no fused append
   unsigned flags;               // MLA_DECODE_* bits of the call
+  const int* worklist;          // tensor-core kernel: unit index per cluster, or null (index order)
 };
 
 // Keys visible to flattened row r = i*H + h of a request holding T keys.

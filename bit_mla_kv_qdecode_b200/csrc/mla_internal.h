@@ -81,6 +81,10 @@ struct DecodeLaunch {
   const void* c_new;
   const void* kr_new;
   int n_new;
+  // tensor-core kernel with a split plan over a multi-wave grid: the order in
+  // which clusters take their units (unit indices, longest first), built on
+  // the device by launch_plan_units in the caller's workspace; null: index order
+  int* worklist;
 };
 
 struct DecodeArgs;
@@ -92,6 +96,11 @@ cudaError_t launch_decode_simt(const DecodeLaunch& L);
 cudaError_t launch_merge2(const float* o_a, const float* l_a, const float* o_b, const float* l_b, int rows,
                           void* out, int out_f32, float* lse, cudaStream_t stream);
 cudaError_t launch_combine(const DecodeLaunch& L);
+// Largest chunk (in pages) a work list handles: the split planner's cap.
+constexpr int kMaxWorklistChunkPages = 128;
+// Fill L.worklist (when set) with the tensor-core kernel's unit indices,
+// longest unit first (one block; launched as a programmatic dependent).
+cudaError_t launch_plan_units(const DecodeLaunch& L, int row_tiles);
 // Returns cudaErrorNotSupported when the tensor-core kernel has no variant for
 // the shape; the caller then uses the SIMT kernel.
 cudaError_t launch_decode_tc(const DecodeLaunch& L);

@@ -204,3 +204,25 @@ def test_hybrid_and_noalloc_argument_errors(lib):
     big = lib.mla_qdecode_noalloc(d, FAKE, FAKE, 4096, FAKE, 262144, FAKE, FAKE, 64, 1, 128, 0.1, 32, FAKE, 0, None,
                                   0, None)
     assert big == E.MLA_ERR_WORKSPACE
+
+
+def test_workspace_holds_the_work_list_of_multi_wave_split_plans():
+    # A split plan for the tensor-core kernel whose units (request, split,
+    # 128-row tile) exceed two waves of the 74 two-CTA cluster slots of a
+    # 148-SM device takes them from a device-built list, one int32 per unit,
+    # placed after the split partials.
+    lib = _lib.load()
+    B, s_q, H, T = 128, 2, 128, 32770
+    n = lib.mla_decode_num_splits(B, s_q, H, T, 0)
+    rows = s_q * H
+    parts = B * n * rows
+    partials = ((parts * 4 + 255) // 256) * 256 + parts * 512 * 4
+    units = B * n * ((rows + 127) // 128)
+    assert n > 1 and units > 148
+    assert lib.mla_decode_workspace_bytes(B, s_q, H, T, 0) == partials + units * 4
+    # one wave or less (here 4 x 32 units), or a small-row plan: no list
+    parts = 4 * 32 * 128
+    assert lib.mla_decode_workspace_bytes(4, 1, 128, 131072, 32) == ((parts * 4 + 255) // 256) * 256 + parts * 2048
+    n16 = lib.mla_decode_num_splits(300, 1, 16, 32768, 0)
+    parts = 300 * n16 * 16
+    assert lib.mla_decode_workspace_bytes(300, 1, 16, 32768, 0) == ((parts * 4 + 255) // 256) * 256 + parts * 2048

@@ -186,3 +186,27 @@ def test_long_request_chunk_cap():
     out, lse = run_decode(case, pool, table_t, num_splits=1)
     err = check(case, out, lse, [0])
     assert err < 1e-3, err
+
+
+def test_skewed_batch_takes_units_longest_first():
+    # One 32,768-key request among 199 short ones (1..399 keys), 128 heads:
+    # the split plan's grid runs in several waves, so the tensor-core kernel
+    # takes its units from the device-built work list, longest first. Every
+    # request matches the oracle, and a second run repeats the first bit for
+    # bit (the order decides only which cluster runs a unit).
+    lens = [32768] + [int(x) for x in np.random.default_rng(11).integers(1, 400, size=199)]
+    w = synth.workload(2).scaled(B=200, H=128, s_q=1)  # INT2 g32 content / INT4 g64 rope
+    case = mc.make_case(w, lens=lens)
+    n = api.mla_decode_num_splits(w.B, 1, w.H, case.max_seq_len, 0)
+    parts = w.B * n * w.H
+    partials = ((parts * 4 + 255) // 256) * 256 + parts * 2048
+    assert n > 1 and api.mla_decode_workspace_bytes(w.B, 1, w.H, case.max_seq_len, 0) == partials + w.B * n * 4
+    pool, table_t, ref, ref_all = mc.fill_pool_with_reference(case, HEADS, all_heads=(0, 7))
+    out, lse = run_decode(case, pool, table_t)
+    assert api.mla_get_device_status() == 0
+    err, lerr = mc.parity(out, lse, ref, heads=HEADS)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
+    err, lerr = mc.parity(out, lse, ref_all)
+    assert err <= mc.RTOL_RMS and lerr <= mc.LSE_ATOL, (err, lerr)
+    again = run_decode(case, pool, table_t)
+    assert torch.equal(out, again[0]) and torch.equal(lse, again[1])
