@@ -67,7 +67,9 @@ struct SplitPlan {
 // (128 query rows of one request and one split) on each 2-CTA cluster slot --
 // or, for at most 16 query rows, one request and split on each of two CTA
 // slots per SM (the small-row kernel) -- and picks the smallest n within 3% of
-// the best, with chunks of at least 4 pages.
+// the best, with chunks of at least 4 pages for the tensor-core kernel (a unit
+// costs it about two pages of set-up and epilogue) and of at least one page
+// for the small-row kernel.
 constexpr int kMaxChunkPages = 128;
 
 SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
@@ -80,7 +82,7 @@ SplitPlan plan_splits(int B, int s_q, int H, int max_seq_len, int requested) {
     const bool small = static_cast<long>(s_q) * H <= mla::kSmallRows;
     const long units = static_cast<long>(std::max(B, 1)) * (small ? 1 : (static_cast<long>(s_q) * H + 127) / 128);
     const long slots = std::max(1, small ? 2 * device_sm_count() : device_sm_count() / 2);
-    const int n_max = std::max(n_min, std::min(pages / 4, 64));
+    const int n_max = std::max(n_min, std::min(small ? pages : pages / 4, 64));
     double best = 1e30;
     n = n_min;
     for (int c = n_min; c <= n_max; ++c) {

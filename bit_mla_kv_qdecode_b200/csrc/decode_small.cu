@@ -190,29 +190,54 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
       const uint32_t* qc = reinterpret_cast<const uint32_t*>(a.q_c);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(a.q_r);
       uint4* qf = reinterpret_cast<uint4*>(smem + Lo::kOffQ);
-      for (int e = tid; e < kGroups * 4 * 32; e += kWarps * 32) {
-        const int g = e / 128, s = (e / 32) & 3, ln = e & 31;
-        const int er = ln >> 2, ekp = ln & 3;
-        const int c = 16 * ekp + 4 * s;  // channel within the group
-        const bool ok0 = er < a.rows, ok1 = er + 8 < a.rows;
-        const size_t q0 = static_cast<size_t>(b) * a.rows + er, q1 = q0 + 8;
-        auto ld = [&](bool ok, size_t q, int cc) -> uint32_t {
-          if (!ok) return 0u;
-          return g < 8 ? __ldg(qc + (q * kDc + 64 * g + cc) / 2) : __ldg(qr + (q * kDr + cc) / 2);
-        };
-        qf[e] = make_uint4(ld(ok0, q0, c), ld(ok1, q1, c), ld(ok0, q0, c + 2), ld(ok1, q1, c + 2));
-      }
-      // per (group, row) sums of q, for the zero-point and code-offset term
-      float* qsum = reinterpret_cast<float*>(smem + Lo::kOffQSum);
-      for (int e = tid; e < kGroups * kRows; e += kWarps * 32) {
-        const int g = e / kRows, row = e % kRows;
-        float acc = 0.0f;
-        if (row < a.rows) {
-          const __nv_bfloat16* q = (g < 8) ? a.q_c + (static_cast<size_t>(b) * a.rows + row) * kDc + 64 * g
-                                           : a.q_r + (static_cast<size_t>(b) * a.rows + row) * kDr;
-          for (int c = 0; c < 64; ++c) acc += __bfloat162float(q[c]);
+      // Every load of the set-up is issued before the first use of any, so
+      // the set-up costs one round trip to memory (it precedes the first page).
+      constexpr int kEntries = kGroups * 4 * 32;
+      constexpr int kPerThread = (kEntries + kWarps * 32 - 1) / (kWarps * 32);
+      uint4 fv[kPerThread];
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k) {
+        const int e = tid + k * kWarps * 32;
+        fv[k] = make_uint4(0, 0, 0, 0);
+        if (e < kEntries) {
+          const int g = e / 128, s = (e / 32) & 3, ln = e & 31;
+          const int er = ln >> 2, ekp = ln & 3;
+          const int c = 16 * ekp + 4 * s;  // channel within the group
+          const bool ok0 = er < a.rows, ok1 = er + 8 < a.rows;
+          const size_t q0 = static_cast<size_t>(b) * a.rows + er, q1 = q0 + 8;
+          auto ld = [&](bool ok, size_t q, int cc) -> uint32_t {
+            if (!ok) return 0u;
+            return g < 8 ? __ldg(qc + (q * kDc + 64 * g + cc) / 2) : __ldg(qr + (q * kDr + cc) / 2);
+          };
+          fv[k] = make_uint4(ld(ok0, q0, c), ld(ok1, q1, c), ld(ok0, q0, c + 2), ld(ok1, q1, c + 2));
         }
-        qsum[e] = acc;
+      }
+      // per (group, row) sums of q, for the zero-point and code-offset term:
+      // a group's 64 channels as eight 16-byte loads
+      const int eg = tid / kRows, erow = tid % kRows;  // threads 0..143: (group, row)
+      const bool sum_ok = tid < kGroups * kRows && erow < a.rows;
+      uint4 qv[8];
+      if (sum_ok) {
+        const uint4* q = reinterpret_cast<const uint4*>(
+            (eg < 8) ? a.q_c + (static_cast<size_t>(b) * a.rows + erow) * kDc + 64 * eg
+                     : a.q_r + (static_cast<size_t>(b) * a.rows + erow) * kDr);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) qv[v] = __ldg(q + v);
+      }
+#pragma unroll
+      for (int k = 0; k < kPerThread; ++k)
+        if (tid + k * kWarps * 32 < kEntries) qf[tid + k * kWarps * 32] = fv[k];
+      if (tid < kGroups * kRows) {
+        float acc = 0.0f;
+        if (sum_ok) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint32_t wv[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc += bf16_lo(wv[e]) + bf16_hi(wv[e]);
+          }
+        }
+        reinterpret_cast<float*>(smem + Lo::kOffQSum)[tid] = acc;  // [group][row]
       }
       named_barrier_compute();
     }
