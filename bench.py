@@ -609,7 +609,14 @@ def main():
     d2h = h_outs[0].numel() * 2 + h_lses[0].numel() * 4
 
     fused = (w.s_q * w.H > 16)  # the small-row kernel takes the append as a separate launch
-    launches_per_step = (1 if fused else 2) + (1 if n_split > 1 else 0)
+    # the tensor-core path plans a multi-wave split grid with one more (single-block)
+    # kernel: its work list, units longest first (the library's rule, restated here)
+    rows = w.s_q * w.H
+    units = w.B * n_split * ((rows + 127) // 128)
+    chunk_pages = -(-((max_len + 63) // 64) // n_split)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    planned = fused and n_split > 1 and chunk_pages <= 128 and units > 2 * (sms // 2)
+    launches_per_step = (1 if fused else 2) + (1 if n_split > 1 else 0) + (1 if planned else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
