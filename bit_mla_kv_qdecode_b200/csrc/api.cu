@@ -239,8 +239,9 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   L.status = status;
   L.stream = c.stream;
 
-  // A fused append runs inside the tensor-core kernel; the other kernels get
-  // the append kernel launched first (lengths here already count the new tokens).
+  // A fused append runs inside the tensor-core and small-row kernels; the
+  // SIMT kernel gets the append kernel launched first (lengths here already
+  // count the new tokens).
   auto append_first = [&]() -> cudaError_t {
     mla::AppendLaunch A{const_cast<void*>(c.pool), c.num_pages, c.block_table, c.max_pages_per_seq, c.seq_lens,
                         c.c_new, c.kr_new, c.B, c.n_new, L.bits_c, L.group_c, L.bits_r, L.group_r,
@@ -249,9 +250,7 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   };
   cudaError_t e = cudaErrorNotSupported;
   if (!(c.flags & MLA_DECODE_FORCE_SIMT)) {
-    if (c.n_new > 0 && mla::decode_small_supported(L)) {
-      if (append_first() != cudaSuccess) return MLA_ERR_CUDA;
-    } else if (c.n_new > 0) {
+    if (c.n_new > 0) {
       L.c_new = c.c_new;
       L.kr_new = c.kr_new;
       L.n_new = c.n_new;
@@ -264,7 +263,7 @@ mla_status run_decode(const DecodeCommon& c, bool quantized, const mla_qcache_de
   }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
-    if (L.n_new > 0) {  // the tensor-core kernel did not take the fused append
+    if (L.n_new > 0) {  // neither the small-row nor the tensor-core kernel took the fused append
       L.n_new = 0;
       if (append_first() != cudaSuccess) return MLA_ERR_CUDA;
     } else if (c.n_new > 0 && (c.flags & MLA_DECODE_FORCE_SIMT)) {

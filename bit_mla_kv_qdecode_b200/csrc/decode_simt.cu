@@ -236,68 +236,67 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
 
 // Split-KV merge: lse = log sum_j exp(lse_j), o = sum_j exp(lse_j - lse) o_j.
 // Splits past the request's last page were never written and are not read;
-// splits that saw no key carry lse_j = -inf and weight 0. One warp per output
-// row: lane l owns the 16-byte pieces l, l+32, l+64, l+96 of the 512 floats,
-// and two splits are loaded per step so that eight loads are in flight.
-// Launched as a programmatic dependent of the decode kernel: it waits for that
-// grid's results before its first read.
+// splits that saw no key carry lse_j = -inf and weight 0. Launched as a
+// programmatic dependent of the decode kernel: it waits for that grid's
+// results before its first read.
 constexpr int kCombineWarps = 8;
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs a) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
+  // One warp per (output row, quarter of its 512 channels): lane l holds
+  // channels [128 q + 4 l, 128 q + 4 l + 4) of every split's partial, and four
+  // splits' loads are in flight at a time, so a row of few splits or a batch
+  // of few rows is not a chain of dependent round trips to memory.
   const int lane = threadIdx.x & 31;
   const long gw = static_cast<long>(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
-  if (gw >= static_cast<long>(a.B) * a.rows) return;
-  const int b = static_cast<int>(gw / a.rows), row = static_cast<int>(gw % a.rows);
+  if (gw >= static_cast<long>(a.B) * a.rows * 4) return;
+  const int quarter = static_cast<int>(gw & 3);
+  const long rw = gw >> 2;
+  const int b = static_cast<int>(rw / a.rows), row = static_cast<int>(rw % a.rows);
   const int T = checked_len(a, b);
   const int pages_b = (T + kPage - 1) / kPage;
   const int n_b = min(a.n_split, (pages_b + a.chunk_pages - 1) / a.chunk_pages);
   const size_t base = static_cast<size_t>(b) * a.n_split;
+  const float* lse_p = a.lse_part + base * a.rows + row;  // split j at [j * rows]
+  const float4* o_p = reinterpret_cast<const float4*>(a.o_part + (base * a.rows + row) * kDc) + quarter * 32 + lane;
+  const size_t o_stride = static_cast<size_t>(a.rows) * (kDc / 4);  // float4 per split
   float m = -CUDART_INF_F;
-  for (int j = lane; j < n_b; j += 32) m = fmaxf(m, a.lse_part[(base + j) * a.rows + row]);
+  for (int j = lane; j < n_b; j += 32) m = fmaxf(m, lse_p[static_cast<size_t>(j) * a.rows]);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float4 acc[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float tot = 0.0f;
   if (m != -CUDART_INF_F) {
-    for (int j = 0; j < n_b; j += 2) {
-      const bool two = j + 1 < n_b;
-      const float w0 = exp2f((a.lse_part[(base + j) * a.rows + row] - m) * kLog2e);
-      const float w1 = two ? exp2f((a.lse_part[(base + j + 1) * a.rows + row] - m) * kLog2e) : 0.0f;
-      const float4* s0 = reinterpret_cast<const float4*>(a.o_part + ((base + j) * a.rows + row) * kDc);
-      const float4* s1 = reinterpret_cast<const float4*>(a.o_part + ((base + j + (two ? 1 : 0)) * a.rows + row) * kDc);
-      float4 v0[4], v1[4];
+    for (int j = 0; j < n_b; j += 4) {
+      float w[4];
+      float4 v[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        v0[q] = s0[lane + 32 * q];
-        v1[q] = two ? s1[lane + 32 * q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 4; ++u) {
+        const bool in = j + u < n_b;
+        w[u] = in ? exp2f((lse_p[static_cast<size_t>(j + u) * a.rows] - m) * kLog2e) : 0.0f;
+        v[u] = in ? o_p[static_cast<size_t>(j + u) * o_stride] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      tot += w0 + w1;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[q].x = fmaf(w1, v1[q].x, fmaf(w0, v0[q].x, acc[q].x));
-        acc[q].y = fmaf(w1, v1[q].y, fmaf(w0, v0[q].y, acc[q].y));
-        acc[q].z = fmaf(w1, v1[q].z, fmaf(w0, v0[q].z, acc[q].z));
-        acc[q].w = fmaf(w1, v1[q].w, fmaf(w0, v0[q].w, acc[q].w));
+      for (int u = 0; u < 4; ++u) {
+        tot += w[u];
+        acc.x = fmaf(w[u], v[u].x, acc.x);
+        acc.y = fmaf(w[u], v[u].y, acc.y);
+        acc.z = fmaf(w[u], v[u].z, acc.z);
+        acc.w = fmaf(w[u], v[u].w, acc.w);
       }
     }
   }
   const float inv = tot > 0.0f ? 1.0f / tot : 0.0f;
   const size_t qrow = static_cast<size_t>(b) * a.rows + row;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 v = make_float4(acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
-    if (a.out_f32) {
-      reinterpret_cast<float4*>(static_cast<float*>(a.out) + qrow * kDc)[lane + 32 * q] = v;
-    } else {
-      const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
-      reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc)[lane + 32 * q] =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
-    }
+  const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (a.out_f32) {
+    reinterpret_cast<float4*>(static_cast<float*>(a.out) + qrow * kDc)[quarter * 32 + lane] = v;
+  } else {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
+    reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc)[quarter * 32 + lane] =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
   }
-  if (lane == 0 && a.lse) a.lse[qrow] = tot > 0.0f ? m + logf(tot) : -CUDART_INF_F;
+  if (quarter == 0 && lane == 0 && a.lse) a.lse[qrow] = tot > 0.0f ? m + logf(tot) : -CUDART_INF_F;
 }
 
 template <class Src>
@@ -362,7 +361,7 @@ cudaError_t launch_decode_simt(const DecodeLaunch& L) {
 
 cudaError_t launch_combine(const DecodeLaunch& L) {
   const DecodeArgs a = make_decode_args(L);
-  const long blocks = (static_cast<long>(a.B) * a.rows + kCombineWarps - 1) / kCombineWarps;
+  const long blocks = (static_cast<long>(a.B) * a.rows * 4 + kCombineWarps - 1) / kCombineWarps;
   if (blocks > 0x7FFFFFFFL) return cudaErrorInvalidValue;
   return launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * kCombineWarps), 0, L.stream,
                           a);

@@ -30,6 +30,7 @@
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
+#include "append_token.cuh"
 #include "mla_common.cuh"
 #include "mla_internal.h"
 #include "sm100_ptx.cuh"
@@ -148,6 +149,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
     ptx::fence_mbar_init_cluster();
   }
   __syncthreads();
+
+  // Fused append (mla_qdecode_fused_append): the step's n_new new tokens are
+  // the last n_new of the T positions. The unit whose key range holds them
+  // quantizes them into the pool (one warp per token, the append kernel's
+  // writer) before it copies any page; the proxy fence and the barrier order
+  // those writes before the bulk copies. Units of other key ranges never read
+  // those bytes.
+  if (a.n_new > 0) {
+    if (T < a.n_new) {
+      if (tid == 0) record_error(a.status, MLA_ERR_INVALID_ARG);
+    } else {
+      const int t_new = T - a.n_new;
+      for (int t = max(t_new, p_begin * kPage) + warp; t < t_end; t += kWarps) {
+        const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t);
+        if (page < 0) {
+          if (lane == 0) record_error(a.status, MLA_ERR_INVALID_ARG);
+          continue;
+        }
+        const size_t src = static_cast<size_t>(b) * a.n_new + (t - t_new);
+        quantize_token_warp<BITS_C, G_C, BITS_R, G_R>(
+            const_cast<uint8_t*>(a.pool) + static_cast<size_t>(page) * G::kPageBytes, t % kPage,
+            a.c_new + src * kDc, a.kr_new + src * kDr, lane);
+      }
+      ptx::fence_proxy_async_global();
+    }
+    __syncthreads();
+  }
 
   // Page k of the unit goes to stage k % kNS. Thread 0 issues pages
   // 0 .. kNS-2 here and page k + kNS - 1 right after page k's named barrier,

@@ -85,7 +85,7 @@ struct DecodeArgs {
   int n_split, chunk_pages;
   int out_f32;
   float scale_log2;          // softmax scale * log2(e)
-  const __nv_bfloat16* c_new;   // fused append: [B, n_new, 512] (tensor-core kernel only)
+  const __nv_bfloat16* c_new;   // fused append: [B, n_new, 512] (tensor-core and small-row kernels)
   const __nv_bfloat16* kr_new;  // [B, n_new, 64]
   int n_new;                    // 0: no fused append
   unsigned flags;               // MLA_DECODE_* bits of the call

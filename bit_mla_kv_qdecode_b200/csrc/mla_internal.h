@@ -75,7 +75,7 @@ struct DecodeLaunch {
   unsigned flags;
   int* status;
   cudaStream_t stream;
-  // fused append (tensor-core kernel only): bf16 c_new [B, n_new, 512] and
+  // fused append (tensor-core and small-row kernels): bf16 c_new [B, n_new, 512] and
   // kr_new [B, n_new, 64] are the last n_new of seq_lens[b] positions; each
   // unit quantizes those in its key range into the pool before reading it
   const void* c_new;

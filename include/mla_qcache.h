@@ -216,12 +216,13 @@ mla_status mla_qdecode(const mla_qcache_desc* desc, const void* pool,
 
 /* One decode step of a speculative-verify / multi-token-prediction loop:
  * the cache append of the step's n_new new tokens followed by mla_qdecode,
- * with the append fused into the decode kernel where the tensor-core kernel
- * runs (each work unit quantizes the new tokens inside its key range into the
- * pool, then reads them back through TMA), which saves the append launch and
- * its latency. Results and pool bytes are those of mla_qcache_append
- * (seq_lens_before = seq_lens - n_new) followed by mla_qdecode; where the
- * fused form does not apply (s_q*H <= 16, MLA_DECODE_FORCE_SIMT) the library
+ * with the append fused into the decode kernel (the tensor-core kernel, and
+ * the small-row kernel for s_q*H <= 16: each work unit quantizes the new
+ * tokens inside its key range into the pool, then copies its pages in), which
+ * saves the append launch and its latency. Results and pool bytes are those of
+ * mla_qcache_append (seq_lens_before = seq_lens - n_new) followed by
+ * mla_qdecode; where the fused form does not apply (MLA_DECODE_FORCE_SIMT, or
+ * a small-row shape in a format the small-row kernel lacks) the library
  * launches the append kernel and then the decode itself.
  * (QuantMLA abstract: tokens are quantized as they are written; the
  * workload's verify step appends s_q tokens per request before the decode.)

@@ -19,7 +19,9 @@ CASES = [
     (2, 32, 4, 64, 128, 2, 2, [2, 65, 66, 300, 4096], 0, 0),       # new tokens straddle a page edge (63, 64)
     (2, 32, 4, 64, 128, 2, 2, [130, 777], 3, 0),                    # split plan: the last split writes
     (4, 64, 4, 64, 64, 3, 3, [5, 200], 1, 0),                       # 192 rows: two row tiles both write
-    (4, 64, 4, 64, 16, 1, 1, [1024, 7], 0, 0),                      # s_q*H <= 16: append kernel, then decode
+    (4, 64, 4, 64, 16, 1, 1, [1024, 7], 0, 0),                      # s_q*H <= 16: fused into the small-row kernel
+    (4, 64, 4, 64, 8, 2, 2, [64, 65, 700], 3, 0),                   # small-row kernel, tokens straddle a page edge
+    (2, 32, 4, 64, 16, 1, 1, [300, 9], 0, 0),                       # s_q*H <= 16, INT2: append kernel, then decode
     (4, 64, 4, 64, 128, 1, 2, [90, 3], 2, MLA_DECODE_FORCE_SIMT),   # SIMT path: append kernel, then decode
 ]
 
