@@ -559,6 +559,7 @@ bool decode_small_supported(const DecodeLaunch& L) {
 }
 
 cudaError_t launch_decode_small(const DecodeLaunch& L) {
+  if (!L.quantized) return launch_decode_small_bf16(L);
   if (!decode_small_supported(L)) return cudaErrorNotSupported;
   return small::launch_t<4, 64, 4, 64>(L);
 }

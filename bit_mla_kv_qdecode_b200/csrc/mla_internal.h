@@ -104,10 +104,13 @@ cudaError_t launch_plan_units(const DecodeLaunch& L, int row_tiles);
 // Returns cudaErrorNotSupported when the tensor-core kernel has no variant for
 // the shape; the caller then uses the SIMT kernel.
 cudaError_t launch_decode_tc(const DecodeLaunch& L);
-// Warp-level MMA kernel for s_q * H <= 16 rows (INT4 g64 content and RoPE);
-// cudaErrorNotSupported for other shapes and formats.
+// Warp-level MMA kernels for s_q * H <= 16 rows (quantized: INT4 g64 content
+// and RoPE; or the BF16 cache); cudaErrorNotSupported for other shapes and formats.
 cudaError_t launch_decode_small(const DecodeLaunch& L);
 bool decode_small_supported(const DecodeLaunch& L);
+// Warp-level MMA kernel for s_q * H <= 16 rows over the BF16 comparison cache.
+cudaError_t launch_decode_small_bf16(const DecodeLaunch& L);
+bool decode_small_bf16_supported(const DecodeLaunch& L);
 // Query rows up to which a decode unit is one CTA of the small-row kernel.
 constexpr int kSmallRows = 16;
 

@@ -89,6 +89,27 @@ def test_bf16_cache_decode(flags, num_splits):
     check(case, out, lse, range(w.B), quantized=False)
 
 
+BF16_SMALL = [
+    # (H, s_q, lens): at most 16 query rows, the warp-level MMA kernel for the BF16 cache
+    (16, 1, [1, 31, 32, 33, 63, 64, 65, 1000]),
+    (8, 2, [2, 65, 300, 4096]),
+    (5, 3, [100, 1, 129]),
+    (1, 1, [33, 640]),
+]
+
+
+@pytest.mark.parametrize("spec", BF16_SMALL)
+@pytest.mark.parametrize("num_splits", [1, 3, 0])
+def test_bf16_cache_small_rows(spec, num_splits):
+    H, s_q, lens = spec
+    w = synth.workload(3).scaled(B=len(lens), H=H, s_q=s_q)
+    case = mc.make_case(w, lens=lens)
+    pool, table_t = mc.fill_pool(case, quantized=False)
+    out, lse = run_decode(case, pool, table_t, num_splits=num_splits, quantized=False)
+    assert api.mla_get_device_status() == 0
+    check(case, out, lse, range(w.B), quantized=False)
+
+
 def test_empty_request_and_length_errors():
     w = synth.workload(1).scaled(B=3)
     case = mc.make_case(w, lens=[0, 70, 0])
@@ -167,7 +188,7 @@ def test_full_size_workloads(idx):
     out, lse = run_decode(case, pool, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16)
     assert api.mla_get_device_status() == 0
     check(case, out, lse, FULL[idx], bf16_out=True)
-    if w.bf16_compare:
+    if w.bf16_compare or w.s_q * w.H <= 16:  # the BF16 comparison decode of these shapes too
         del pool
         pool_b, _ = mc.fill_pool(case, quantized=False)
         out, lse = run_decode(case, pool_b, table_t, num_splits=w.num_splits, out_dtype=torch.bfloat16,
