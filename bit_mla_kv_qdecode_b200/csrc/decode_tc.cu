@@ -27,6 +27,14 @@
 // + P_hi*C_lo. All accumulation is fp32 in TMEM. This keeps the output within
 // 2e-3 of its RMS of the exact float64 result; single bf16 operands would not.
 //
+// Pipeline. A chunk's operand tile (C_hi, C_lo of this CTA's 288 channels,
+// 36 KB) is held from its dequantization until its PV MMAs finish; four
+// operand stages, two code stages and one weight tile (rewritten only after
+// the previous chunk's PV) fit the shared memory. The softmax step of chunk
+// j reads the peer's partial scores of chunk j-1, sends this CTA's partial of
+// chunk j, and only then finishes chunk j-1: the copy to the peer is in
+// flight during that work (measured 7-12 % faster than finishing chunk j-1
+// first, once the fourth operand stage relieved the stage ring).
 // Warp roles (512 threads):
 //   warp 0      TMA producer: packed codes + metadata of 32-token chunks
 //   warp 1      TMEM owner; issues the QK MMAs of even chunks
@@ -66,8 +74,9 @@ constexpr int kRows = 128;            // query rows per unit (MMA M)
 constexpr int kHalfC = 256;           // content channels per CTA
 constexpr int kHalfR = 32;            // rope channels per CTA
 constexpr int kKChunks = (kHalfC + kHalfR) / 8;  // 36 eight-channel chunks per token
-constexpr int kNC = 3;                // operand-tile stages
-constexpr int kNS = 4;                // TMA code stages
+constexpr int kNC = 4;                // operand-tile stages
+constexpr int kNS = 2;                // TMA code stages
+constexpr int kBarCode = kNC > kNS ? kNC : kNS;  // code_full entries (the BF16 cache uses one per operand stage)
 static_assert(kChunk == 32, "the PV issue sequence covers two 16-token K-steps");
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (weights stay <= 2^8)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -100,15 +109,15 @@ constexpr int kXBuf = 2 * kXHalf;
 constexpr int kCodeCC = 4096;                      // content codes half (32 tokens x <=128 B)
 constexpr int kCodeRC = 1024;                      // rope codes (32 tokens x <=32 B)
 constexpr int kCodeCM = 1024;                      // content meta half (32 tokens x <=32 B)
-constexpr int kCodeStage = 8192;                   // each sub-buffer 1024-aligned inside
+constexpr int kCodeStage = 7168;                   // content codes 1024-aligned at its start; <= 6,400 B used
 constexpr int kOffC = 0;
 constexpr int kOffP = kOffC + kNC * kCStage;
-constexpr int kOffX = kOffP + 2 * 2 * kPTile;
+constexpr int kOffX = kOffP + 2 * kPTile;  // one weight tile (hi, lo): rewritten only after PV of the previous chunk
 constexpr int kOffCode = kOffX + 2 * kXBuf;
 constexpr int kOffBar = kOffCode + kNS * kCodeStage + kRows * kHalfR * 2;
 constexpr int kOffQR = kOffCode + kNS * kCodeStage;  // rope part of Q: 128 rows x 32 bf16, core matrices
 constexpr int kQRBytes = kRows * kHalfR * 2;
-constexpr int kNumBars = 2 * kNS + 3 * kNC + 16 + 12;
+constexpr int kNumBars = kBarCode + kNS + 3 * kNC + 16 + 12;
 constexpr int kOffMisc = kOffQR + kQRBytes + kNumBars * 8;
 constexpr int kOffRed = kOffMisc + 64;  // row-pair exchange: [2 parity][2 halves][128] maxima, [2][128] sums
 constexpr int kSmemBytes = kOffRed + (2 * 2 * kRows + 2 * kRows) * 4;
@@ -129,15 +138,15 @@ struct TmapSet {
 };
 
 struct Bars {
-  uint64_t* code_full;   // [kNS] TMA -> dequant
+  uint64_t* code_full;   // [kBarCode] TMA -> dequant (quantized: per code stage; BF16: per operand stage)
   uint64_t* code_empty;  // [kNS] dequant -> TMA
   uint64_t* c_full;      // [kNC] dequant -> MMA: channel chunks 0-15 of the stage written
   uint64_t* c_full2;     // [kNC] dequant -> MMA: chunks 16-35 written
   uint64_t* c_empty;     // [kNC] MMA (after PV) -> dequant
   uint64_t* s_full;      // [2] MMA (QK) -> softmax
   uint64_t* s_empty;     // [2] softmax read S -> MMA
-  uint64_t* p_full;      // [2] softmax P tile + O rescale -> MMA
-  uint64_t* p_empty;     // [2] MMA (PV) -> softmax
+  uint64_t* p_full;      // [1] softmax P tile + O rescale -> MMA (one tile buffer; slot 1 unused)
+  uint64_t* p_empty;     // [1] MMA (PV) -> softmax
   uint64_t* x_full;      // [2] peer wrote its partial scores into my exchange buffer
   uint64_t* q_full;      // [1] Q in TMEM
   uint64_t* o_full;      // [1] all PV MMAs of the unit done
@@ -151,10 +160,10 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   uint64_t* b = reinterpret_cast<uint64_t*>(smem + kOffBar);
   Bars r;
   r.code_full = b;
-  r.code_empty = b + kNS;
-  r.c_full = b + 2 * kNS;
-  r.c_empty = b + 2 * kNS + kNC;
-  uint64_t* p = b + 2 * kNS + 2 * kNC;
+  r.code_empty = b + kBarCode;
+  r.c_full = b + kBarCode + kNS;
+  r.c_empty = b + kBarCode + kNS + kNC;
+  uint64_t* p = b + kBarCode + kNS + 2 * kNC;
   r.s_full = p;
   r.s_empty = p + 2;
   r.p_full = p + 4;
@@ -166,7 +175,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t* smem) {
   r.qk_drain2 = p + 15;
   r.pair_max = p + 16;
   r.pair_sum = p + 24;
-  r.c_full2 = p + 28;
+  r.c_full2 = p + 28;  // [kNC]
   return r;
 }
 
@@ -245,6 +254,21 @@ __device__ __forceinline__ void dequant_split8(uint32_t w, float2 s2, float2 z2,
   lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Multiply one TMEM lane's 128 fp32 output columns at taddr by f
+// (warp-collective: each lane scales its own row). Out of line: it runs
+// rarely, and inlined its 32-register buffer would crowd the softmax loop.
+__device__ __noinline__ void rescale_cols(uint32_t taddr, float f) {
+#pragma unroll 1
+  for (int c = 0; c < kHalfC / 64; ++c) {
+    uint32_t ov[32];
+    ptx::tmem_ld32(taddr + c * 32, ov);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
+    ptx::tmem_st32(taddr + c * 32, ov);
+  }
+}
+
 __device__ __forceinline__ void fail(const DecodeArgs& a, volatile int* abort_flag) {
   record_error(a.status, MLA_ERR_TIMEOUT);
   *abort_flag = 1;
@@ -268,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const Bars bars = carve_bars(smem);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
-  volatile int* stage_page = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);  // [kNS]
+  volatile int* stage_page = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);  // [kBarCode]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t crank = ptx::cluster_ctarank();
@@ -318,10 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   // ---- setup ----
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
-      ptx::mbar_init(&bars.code_full[i], 1);
-      ptx::mbar_init(&bars.code_empty[i], 128);
-    }
+    for (int i = 0; i < kBarCode; ++i) ptx::mbar_init(&bars.code_full[i], 1);
+    for (int i = 0; i < kNS; ++i) ptx::mbar_init(&bars.code_empty[i], 128);
     for (int i = 0; i < kNC; ++i) {
       ptx::mbar_init(&bars.c_full[i], 128);
       ptx::mbar_init(&bars.c_full2[i], 128);
@@ -514,8 +536,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                    kBF16 ? kBfChunkStride : kCChunkStride);
       bool ok = true;
       for (int j = 0; j < n_chunks; ++j) {
-        const int pb = j & 1, cs = j % kNC;
-        if (!ptx::mbar_wait(&bars.p_full[pb], (j >> 1) & 1, abort_flag, wlim)) {
+        const int cs = j % kNC;
+        if (!ptx::mbar_wait(&bars.p_full[0], j & 1, abort_flag, wlim)) {
           ok = false;
           break;
         }
@@ -523,7 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // Straight-line issue: the issuing thread runs no per-instruction
         // address or predicate arithmetic between the MMAs (measured: such
         // work between two tcgen05.mma instructions slows their issue).
-        const uint64_t ap = a0 + static_cast<uint64_t>((pb * 2 * kPTile) >> 4);
+        const uint64_t ap = a0;
         const uint64_t bc = b0 + static_cast<uint64_t>((cs * kCStage) >> 4);
         const uint64_t ap_lo = ap + static_cast<uint64_t>(kPTile >> 4);    // P_lo
         const uint64_t bc_lo = bc + static_cast<uint64_t>(kCLoOff >> 4);   // C_lo
@@ -540,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ptx::mma_ss(o, ap, bc_lo, idesc, 1u);
           ptx::mma_ss(o, ap + kK1, bc_lo + kK1, idesc, 1u);
         }
-        ptx::mma_commit(&bars.p_empty[pb]);
+        ptx::mma_commit(&bars.p_empty[0]);
         ptx::mma_commit(&bars.c_empty[cs]);
       }
       if (!ok) fail(a, abort_flag);
@@ -694,13 +716,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int prev_page = -1;
 
     // Chunk jj's weight tile (my 16 tokens of this row) -> shared memory,
-    // once PV of chunk jj-2 released the buffer. False when the wait gave up.
+    // once PV of chunk jj-1 has released the one tile buffer (the phase waited
+    // for is the latest: PV of chunk jj needs this tile first, so no later
+    // phase can have completed). False when the wait gave up.
     auto store_weights = [&](int jj, const uint32_t (&ph)[8], const uint32_t (&pl)[8]) -> bool {
-      const int pb = jj & 1;
-      if (jj >= 2 &&
-          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[pb], ((jj - 2) >> 1) & 1, abort_flag, wlim)))
+      if (jj >= 1 &&
+          !__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[0], (jj - 1) & 1, abort_flag, wlim)))
         return false;
-      uint8_t* pt = smem + kOffP + pb * 2 * kPTile + (i >> 3) * 512 + (i & 7) * 16;
+      uint8_t* pt = smem + kOffP + (i >> 3) * 512 + (i & 7) * 16;
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int kc = 2 * h + kk;
@@ -718,60 +741,96 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       // rescale my half of this row of O in TMEM (warp-collective: lanes that
       // do not need it multiply by 1); O must be quiescent: PV of chunk jj-1 done
       if (__any_sync(kFull, rescale && o_live)) {
-        if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[(jj - 1) & 1], ((jj - 1) >> 1) & 1, abort_flag,
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.p_empty[0], (jj - 1) & 1, abort_flag,
                                               wlim)))
           return false;
         ptx::tc_fence_after();
-        const float f = (rescale && o_live) ? alpha : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < kHalfC / 64; ++c) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * f);
-          ptx::tmem_st32(lane_base + kTmemO + h * (kHalfC / 2) + c * 32, ov);
-        }
+        rescale_cols(lane_base + kTmemO + h * (kHalfC / 2), (rescale && o_live) ? alpha : 1.0f);
         ptx::tmem_st_wait();
       }
       o_live = true;
       if (fence) ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars.p_full[jj & 1]);
+      ptx::mbar_arrive(&bars.p_full[0]);
       return true;
     };
 
-    // Step j: the scores and weight tile of chunk j-1 (it needs the peer's
-    // partial, sent one step earlier), then the read and send of this CTA's
-    // partial of chunk j. The quantized path releases chunk j-1's tile to PV
-    // only after the send (whose proxy fence then covers the tile too), so
-    // the release and any O rescale fill the time the copy is in flight; the
-    // BF16 path releases it first, since its operand stages wait on PV and
-    // then on HBM.
+    // Step j: first the peer's partial scores of chunk j-1 (sent one step
+    // earlier) into registers, then the read and send of this CTA's partial
+    // of chunk j (staged in the exchange slot just read), then the softmax of
+    // chunk j-1 and its weight tile: the copy to the peer is in flight while
+    // this thread finishes the previous chunk.
     for (int j = 0; j <= n_chunks && ok; ++j) {
-      uint32_t ph[8], pl[8];
-      float alpha = 1.0f;
-      bool rescale = false;
+      float pvv[16];
       if (j >= 1) {
         const int jj = j - 1, pb = jj & 1;
-        const int t0 = t_begin + jj * kChunk;
         if (!__all_sync(kFull, ptx::mbar_wait(&bars.x_full[pb], (jj >> 1) & 1, abort_flag, wlim))) {
           ok = false;
           break;
         }
         const float4* xr = reinterpret_cast<const float4*>(smem + kOffX + pb * kXBuf + h * kXHalf + i * kXRowBytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 pv = xr[k ^ ((i >> 1) & 3)];
+          pvv[4 * k] = pv.x; pvv[4 * k + 1] = pv.y; pvv[4 * k + 2] = pv.z; pvv[4 * k + 3] = pv.w;
+        }
+      }
+      uint32_t cur[16];
+      int cur_page = -1;
+      if (j < n_chunks) {
+        const int sb = j & 1;
+        // block-table entry of chunk j, checked one step later: issued before the wait to hide the load
+        cur_page = table_entry(a.table, a.max_pages, b, t_begin + j * kChunk);
+        // wait results are made warp-uniform: the TMEM loads below are warp-collective
+        if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, wlim))) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + 16 * h, cur);
+        if (n_terms_qk == 2) {  // add the C_lo half of the score tile, 8 columns at a time
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            uint32_t lo[8];
+            ptx::tmem_ld8(lane_base + kTmemS + sb * 2 * kChunk + kChunk + 16 * h + 8 * g, lo);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              cur[8 * g + k] = __float_as_uint(__uint_as_float(cur[8 * g + k]) + __uint_as_float(lo[k]));
+          }
+        }
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars.s_empty[sb]);
+        // Send my partial scores to the peer, staged in the other exchange
+        // slot, whose segment for my row and half I read above (chunk j-1);
+        // the peer writes that slot again (chunk j+1) only after this copy
+        // has landed, and I restage it only after that.
+        const int blk = h * kXHalf + quarter * kXWarpBlock;
+        uint8_t* stage = smem + kOffX + (sb ^ 1) * kXBuf + h * kXHalf + i * kXRowBytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(stage + 16 * (k ^ ((i >> 1) & 3))) = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (i == 0 && h == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kXBuf);
+        if (lane == 0)
+          ptx::bulk_copy_to_peer(xbuf_peer + sb * kXBuf + blk, smem + kOffX + (sb ^ 1) * kXBuf + blk, kXWarpBlock,
+                                 xfull_peer + sb * 8);
+      }
+      if (j >= 1) {
+        const int jj = j - 1, pb = jj & 1;
+        const int t0 = t_begin + jj * kChunk;
+        uint32_t ph[8], pl[8];
+        float alpha = 1.0f;
+        bool rescale = false;
         // full score = my partial + peer partial, then * scale * log2(e)
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
         float2 sp[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float4 pv = xr[k ^ ((i >> 1) & 3)];
-          sp[2 * k] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k]), __uint_as_float(prev[4 * k + 1])),
-                                            make_float2(pv.x, pv.y)), sc2);
-          sp[2 * k + 1] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[4 * k + 2]),
-                                                            __uint_as_float(prev[4 * k + 3])),
-                                                make_float2(pv.z, pv.w)), sc2);
-        }
+        for (int k = 0; k < 8; ++k)
+          sp[k] = __fmul2_rn(__fadd2_rn(make_float2(__uint_as_float(prev[2 * k]), __uint_as_float(prev[2 * k + 1])),
+                                        make_float2(pvv[2 * k], pvv[2 * k + 1])), sc2);
         const int lim = (page_valid(prev_page, a.num_pages) ? min(L, t_end) - t0 : 0) - 16 * h;  // visible columns in my half
         if (lim < 16) {
 #pragma unroll
@@ -826,63 +885,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < w; ++k) ps[k] = __fadd2_rn(ps[k], ps[k + w]);
         l_sum = l_sum * alpha + (ps[0].x + ps[0].y);
-
-      }
-      if (j >= 1 && !store_weights(j - 1, ph, pl)) {
-        ok = false;
-        break;
-      }
-      if constexpr (kBF16) {  // operands arrive straight from HBM: release PV as early as possible
-        if (j >= 1 && !release_weights(j - 1, alpha, rescale, true)) {
-          ok = false;
-          break;
-        }
-      }
-      uint32_t cur[16];
-      int cur_page = -1;
-      if (j < n_chunks) {
-        const int sb = j & 1;
-        // block-table entry of chunk j, checked one step later: issued before the wait to hide the load
-        cur_page = table_entry(a.table, a.max_pages, b, t_begin + j * kChunk);
-        // wait results are made warp-uniform: the TMEM loads below are warp-collective
-        if (!__all_sync(kFull, ptx::mbar_wait(&bars.s_full[sb], (j >> 1) & 1, abort_flag, wlim))) {
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-        ptx::tmem_ld16(lane_base + kTmemS + sb * 2 * kChunk + 16 * h, cur);
-        if (n_terms_qk == 2) {  // add the C_lo half of the score tile, 8 columns at a time
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            uint32_t lo[8];
-            ptx::tmem_ld8(lane_base + kTmemS + sb * 2 * kChunk + kChunk + 16 * h + 8 * g, lo);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              cur[8 * g + k] = __float_as_uint(__uint_as_float(cur[8 * g + k]) + __uint_as_float(lo[k]));
-          }
-        }
-        ptx::tmem_ld_wait();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars.s_empty[sb]);
-        // Send my partial scores to the peer. They are staged in the other
-        // exchange slot, whose segment for my row and half I finished reading
-        // above (chunk j-1); the peer writes that slot again (chunk j+1) only
-        // after this copy has landed, and I restage it only after that.
-        const int blk = h * kXHalf + quarter * kXWarpBlock;
-        uint8_t* stage = smem + kOffX + (sb ^ 1) * kXBuf + h * kXHalf + i * kXRowBytes;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          *reinterpret_cast<uint4*>(stage + 16 * (k ^ ((i >> 1) & 3))) = make_uint4(cur[4 * k], cur[4 * k + 1], cur[4 * k + 2], cur[4 * k + 3]);
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (i == 0 && h == 0) ptx::mbar_arrive_expect_tx(&bars.x_full[sb], kXBuf);
-        if (lane == 0)
-          ptx::bulk_copy_to_peer(xbuf_peer + sb * kXBuf + blk, smem + kOffX + (sb ^ 1) * kXBuf + blk, kXWarpBlock,
-                                 xfull_peer + sb * 8);
-      }
-      if constexpr (!kBF16) {
-        if (j >= 1 && !release_weights(j - 1, alpha, rescale, j == n_chunks)) {
+        if (!store_weights(jj, ph, pl) || !release_weights(jj, alpha, rescale, true)) {
           ok = false;
           break;
         }
