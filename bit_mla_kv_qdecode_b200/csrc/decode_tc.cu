@@ -699,14 +699,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(bars.q_full);
     }
 
-    // Score exchange. Step j first finishes chunk j-1 (its peer partial was
-    // sent at the end of the previous step), then reads this CTA's partial
-    // S_j from TMEM, stages it in the exchange slot it has just read, and
-    // each warp bulk-copies its 32 rows x 16 columns to the same place in the
-    // peer's slot j&1 (the copy engine completes the bytes on the peer's
-    // x_full). No release handshake is needed: the peer sends chunk j+1 into
-    // the staging slot only after it received chunk j, i.e. after this
-    // copy has read the stage.
+    // Score exchange. Each CTA reads its partial S_j from TMEM, stages it in
+    // its own exchange slot (j+1)&1 (whose chunk j-1 entries it has just
+    // read), and each warp bulk-copies its 32 rows x 16 columns to the same
+    // place in the peer's slot j&1 (the copy engine completes the bytes on
+    // the peer's x_full). No release handshake is needed: the peer sends
+    // chunk j+1 into the staging slot only after it received chunk j, i.e.
+    // after this copy has read the stage.
     const uint32_t xbuf_peer = ptx::mapa(ptx::smem_u32(smem + kOffX), peer);
     const uint32_t xfull_peer = ptx::mapa(ptx::smem_u32(bars.x_full), peer);
     float m_used = -CUDART_INF_F, l_sum = 0.0f;  // l_sum: this half's columns only
