@@ -239,64 +239,94 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
 // splits that saw no key carry lse_j = -inf and weight 0. Launched as a
 // programmatic dependent of the decode kernel: it waits for that grid's
 // results before its first read.
+//
+// A warp merges 512 / kParts channels of one output row: lane l holds the
+// 16-byte pieces 32 q + l (q < 4 / kParts) of its part in every split. The
+// loads of four splits (their lse and their pieces) are issued together and
+// merged online against a running maximum, so a row of up to four splits
+// costs one round trip to memory. kParts = 4 spreads a small batch over more
+// warps; large batches take a whole row per warp (fewer, longer warps).
 constexpr int kCombineWarps = 8;
+constexpr int kCombineGroup = 4;  // splits in flight per warp
+constexpr long kCombineSmallRows = 148 * 16;  // output rows below which a row is split over four warps
+template <int kParts>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs a) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
-  // One warp per (output row, quarter of its 512 channels): lane l holds
-  // channels [128 q + 4 l, 128 q + 4 l + 4) of every split's partial, and four
-  // splits' loads are in flight at a time, so a row of few splits or a batch
-  // of few rows is not a chain of dependent round trips to memory.
+  constexpr int kVec = 4 / kParts;  // 16-byte pieces per lane and split
   const int lane = threadIdx.x & 31;
   const long gw = static_cast<long>(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
-  if (gw >= static_cast<long>(a.B) * a.rows * 4) return;
-  const int quarter = static_cast<int>(gw & 3);
-  const long rw = gw >> 2;
+  if (gw >= static_cast<long>(a.B) * a.rows * kParts) return;
+  const int part = static_cast<int>(gw % kParts);
+  const long rw = gw / kParts;
   const int b = static_cast<int>(rw / a.rows), row = static_cast<int>(rw % a.rows);
   const int T = checked_len(a, b);
   const int pages_b = (T + kPage - 1) / kPage;
   const int n_b = min(a.n_split, (pages_b + a.chunk_pages - 1) / a.chunk_pages);
   const size_t base = static_cast<size_t>(b) * a.n_split;
   const float* lse_p = a.lse_part + base * a.rows + row;  // split j at [j * rows]
-  const float4* o_p = reinterpret_cast<const float4*>(a.o_part + (base * a.rows + row) * kDc) + quarter * 32 + lane;
+  const float4* o_p =
+      reinterpret_cast<const float4*>(a.o_part + (base * a.rows + row) * kDc) + part * 32 * kVec + lane;
   const size_t o_stride = static_cast<size_t>(a.rows) * (kDc / 4);  // float4 per split
-  float m = -CUDART_INF_F;
-  for (int j = lane; j < n_b; j += 32) m = fmaxf(m, lse_p[static_cast<size_t>(j) * a.rows]);
+  float m = -CUDART_INF_F, tot = 0.0f;
+  float4 acc[kVec];
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float tot = 0.0f;
-  if (m != -CUDART_INF_F) {
-    for (int j = 0; j < n_b; j += 4) {
-      float w[4];
-      float4 v[4];
+  for (int q = 0; q < kVec; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < n_b; j += kCombineGroup) {
+    float l[kCombineGroup];
+    float4 v[kCombineGroup][kVec];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool in = j + u < n_b;
-        w[u] = in ? exp2f((lse_p[static_cast<size_t>(j + u) * a.rows] - m) * kLog2e) : 0.0f;
-        v[u] = in ? o_p[static_cast<size_t>(j + u) * o_stride] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kCombineGroup; ++u) {
+      const bool in = j + u < n_b;
+      l[u] = in ? lse_p[static_cast<size_t>(j + u) * a.rows] : -CUDART_INF_F;
+#pragma unroll
+      for (int q = 0; q < kVec; ++q)
+        v[u][q] = in ? o_p[static_cast<size_t>(j + u) * o_stride + 32 * q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mg = l[0];
+#pragma unroll
+    for (int u = 1; u < kCombineGroup; ++u) mg = fmaxf(mg, l[u]);
+    if (mg == -CUDART_INF_F) continue;  // no split of this group saw a key (same values in every lane)
+    if (mg > m) {  // the running maximum moves: rescale what is merged so far
+      const float f = (m == -CUDART_INF_F) ? 0.0f : exp2f((m - mg) * kLog2e);
+      tot *= f;
+#pragma unroll
+      for (int q = 0; q < kVec; ++q) {
+        acc[q].x *= f;
+        acc[q].y *= f;
+        acc[q].z *= f;
+        acc[q].w *= f;
       }
+      m = mg;
+    }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        tot += w[u];
-        acc.x = fmaf(w[u], v[u].x, acc.x);
-        acc.y = fmaf(w[u], v[u].y, acc.y);
-        acc.z = fmaf(w[u], v[u].z, acc.z);
-        acc.w = fmaf(w[u], v[u].w, acc.w);
+    for (int u = 0; u < kCombineGroup; ++u) {
+      const float w = exp2f((l[u] - m) * kLog2e);  // lse -inf -> 0
+      tot += w;
+#pragma unroll
+      for (int q = 0; q < kVec; ++q) {
+        acc[q].x = fmaf(w, v[u][q].x, acc[q].x);
+        acc[q].y = fmaf(w, v[u][q].y, acc[q].y);
+        acc[q].z = fmaf(w, v[u][q].z, acc[q].z);
+        acc[q].w = fmaf(w, v[u][q].w, acc[q].w);
       }
     }
   }
   const float inv = tot > 0.0f ? 1.0f / tot : 0.0f;
   const size_t qrow = static_cast<size_t>(b) * a.rows + row;
-  const float4 v = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (a.out_f32) {
-    reinterpret_cast<float4*>(static_cast<float*>(a.out) + qrow * kDc)[quarter * 32 + lane] = v;
-  } else {
-    const __nv_bfloat162 h0 = __floats2bfloat162_rn(v.x, v.y), h1 = __floats2bfloat162_rn(v.z, v.w);
-    reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc)[quarter * 32 + lane] =
-        make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+#pragma unroll
+  for (int q = 0; q < kVec; ++q) {
+    const int piece = part * 32 * kVec + 32 * q + lane;
+    const float4 r = make_float4(acc[q].x * inv, acc[q].y * inv, acc[q].z * inv, acc[q].w * inv);
+    if (a.out_f32) {
+      reinterpret_cast<float4*>(static_cast<float*>(a.out) + qrow * kDc)[piece] = r;
+    } else {
+      const __nv_bfloat162 h0 = __floats2bfloat162_rn(r.x, r.y), h1 = __floats2bfloat162_rn(r.z, r.w);
+      reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + qrow * kDc)[piece] =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+    }
   }
-  if (quarter == 0 && lane == 0 && a.lse) a.lse[qrow] = tot > 0.0f ? m + logf(tot) : -CUDART_INF_F;
+  if (part == 0 && lane == 0 && a.lse) a.lse[qrow] = tot > 0.0f ? m + logf(tot) : -CUDART_INF_F;
 }
 
 template <class Src>
@@ -361,10 +391,14 @@ cudaError_t launch_decode_simt(const DecodeLaunch& L) {
 
 cudaError_t launch_combine(const DecodeLaunch& L) {
   const DecodeArgs a = make_decode_args(L);
-  const long blocks = (static_cast<long>(a.B) * a.rows * 4 + kCombineWarps - 1) / kCombineWarps;
+  const long rows = static_cast<long>(a.B) * a.rows;
+  // fewer rows than 16 whole-row warps for each of 148 SMs: split each row over four warps
+  const bool quarter = rows < kCombineSmallRows;
+  const long blocks = (rows * (quarter ? 4 : 1) + kCombineWarps - 1) / kCombineWarps;
   if (blocks > 0x7FFFFFFFL) return cudaErrorInvalidValue;
-  return launch_dependent(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * kCombineWarps), 0, L.stream,
-                          a);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(32 * kCombineWarps);
+  return quarter ? launch_dependent(combine_kernel<4>, grid, block, 0, L.stream, a)
+                 : launch_dependent(combine_kernel<1>, grid, block, 0, L.stream, a);
 }
 
 }  // namespace mla

@@ -182,10 +182,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
   // when every warp is past the output MMAs of page k - 1, the last reader of
   // that stage. A missing page arrives without bytes; its keys are masked.
   int n_issued = 0;
-  auto issue_page = [&](int k) {
+  auto entry_of = [&](int k) { return k < n_pages ? table_entry(a.table, a.max_pages, b, (p_begin + k) * kPage) : -1; };
+  auto issue_page = [&](int k, int page) {  // page: the block-table entry of unit page k
     if (k >= n_pages) return;
     const int s = k % kNS;
-    const int page = table_entry(a.table, a.max_pages, b, (p_begin + k) * kPage);
     if (page_valid(page, a.num_pages)) {
       stage_page[s] = page;
       ptx::mbar_arrive_expect_tx(&full[s], G::kPageBytes);
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
     n_issued = k + 1;
   };
   if (tid == 0)
-    for (int k = 0; k < kNS - 1; ++k) issue_page(k);
+    for (int k = 0; k < kNS - 1; ++k) issue_page(k, entry_of(k));
 
   {
     // =========================== compute warps ===========================
@@ -281,6 +281,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
 
     for (int k = 0; k < n_pages; ++k) {
       const int s = k % kNS, pb = k & 1;
+      // the entry of the page issued after this page's barrier, loaded now so
+      // that the issuing thread does not hold the next barrier up
+      const int next_entry = tid == 0 ? entry_of(k + kNS - 1) : -1;
       // on a timeout the loop runs on (every warp keeps the same barrier
       // sequence) with the abort flag set, so later waits return at once
       if (!ptx::mbar_wait(&full[s], (k / kNS) & 1, abort_flag, kWaitLimitNs)) {
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
         mt[(r + 8) * kWarps + w] = mw[1];
       }
       named_barrier_compute();
-      if (tid == 0) issue_page(k + kNS - 1);
+      if (tid == 0) issue_page(k + kNS - 1, next_entry);
 
       // ---- new running maximum; rescale O and the row sums when it moved ----
       float mwr[2][kWarps];
@@ -368,11 +371,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
         mwr[i][4] = v.x; mwr[i][5] = v.y; mwr[i][6] = v.z; mwr[i][7] = v.w;
       }
       float mnew[2], alpha[2];
+      bool uniform = true;  // every warp took its weights against the new maximum (the common case)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         mnew[i] = m_run[i];
 #pragma unroll
         for (int v = 0; v < kWarps; ++v) mnew[i] = fmaxf(mnew[i], mwr[i][v]);
+#pragma unroll
+        for (int v = 0; v < kWarps; ++v) uniform &= mwr[i][v] == mnew[i];
         alpha[i] = (mnew[i] == -CUDART_INF_F) ? 1.0f : exp2f(m_run[i] - mnew[i]);
         const float own = (mw[i] == -CUDART_INF_F) ? 0.0f : exp2f(mw[i] - mnew[i]);
         l_acc[i] = l_acc[i] * alpha[i] + l_own[i] * own;
@@ -388,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
           o[j][3] *= alpha[1];
         }
       }
+      const bool rescale_w = __any_sync(kFull, !uniform);
 
       // ---- O[16 rows, group w] += sum_t p_t c_hat_t over the page ----
       // Block j, column n holds channel 64w + 8n + j: lane (r, kp) supplies
@@ -402,15 +409,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
                         *reinterpret_cast<const float2*>(ptile + (r + 8) * kPRow + ta * 4),
                         *reinterpret_cast<const float2*>(ptile + r * kPRow + tb * 4),
                         *reinterpret_cast<const float2*>(ptile + (r + 8) * kPRow + tb * 4)};
-        float fq[4];
-        bool scale_w = false;
+        if (rescale_w) {  // some warp's maximum differs from the new one: scale its weights
+          float fq[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float mq = mwr[q & 1][2 * ks + (q >> 1)];
-          fq[q] = (mq == -CUDART_INF_F) ? 0.0f : exp2f(mq - mnew[q & 1]);
-          scale_w |= fq[q] != 1.0f;
-        }
-        if (__any_sync(kFull, scale_w)) {
+          for (int q = 0; q < 4; ++q) {
+            const float mq = mwr[q & 1][2 * ks + (q >> 1)];
+            fq[q] = (mq == -CUDART_INF_F) ? 0.0f : exp2f(mq - mnew[q & 1]);
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             pw[q].x *= fq[q];

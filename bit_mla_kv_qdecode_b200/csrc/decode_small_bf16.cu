@@ -129,11 +129,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
   // weights are 0, and 0 times stale bytes must not meet a NaN). The zeroing
   // stores come before the arrive that opens the stage's phase.
   int n_issued = 0;
-  auto issue_stage = [&](int k) {  // warp 0, all lanes
+  auto page_of = [&](int k) {
+    return k < n_st ? lookup_page(a.table, a.max_pages, a.num_pages, b, t_begin + k * kTok) : -1;
+  };
+  auto issue_stage = [&](int k, int page) {  // warp 0, all lanes; page: lookup_page of stage k
     if (k >= n_st) return;
     const int s = k % kNS;
     const int t0 = t_begin + k * kTok;
-    const int page = lookup_page(a.table, a.max_pages, a.num_pages, b, t0);
     const int n_valid = page >= 0 ? min(kTok, t_end - t0) : 0;
     uint8_t* row = smem + s * kStage + lane * kRowStride;
     if (lane >= n_valid) {
@@ -158,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
     n_issued = k + 1;
   };
   if (warp == 0)
-    for (int k = 0; k < kNS - 1; ++k) issue_stage(k);
+    for (int k = 0; k < kNS - 1; ++k) issue_stage(k, page_of(k));
 
   const int r = lane >> 2, kp = lane & 3;  // MMA fragment coordinates: row group, k pair
   const bool row_ok0 = r < a.rows, row_ok1 = r + 8 < a.rows;
@@ -210,6 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
 
   for (int k = 0; k < n_st; ++k) {
     const int s = k % kNS;
+    // the page of the stage issued after this stage's weights, loaded now so
+    // that warp 0 does not hold the next barrier up
+    const int next_page = warp == 0 ? page_of(k + kNS - 1) : -1;
     // on a timeout the loop runs on (every warp keeps the same barrier
     // sequence) with the abort flag set, so later waits return at once
     if (!ptx::mbar_wait(&full[s], (k / kNS) & 1, abort_flag, kWaitLimitNs)) {
@@ -224,16 +229,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     {
       // ldmatrix rows: keys 8nt + (lane & 7); matrices (K-step, channels
-      // 0-7), (K-step, 8-15), (next K-step, 0-7), (next K-step, 8-15)
+      // 0-7), (K-step, 8-15), (next K-step, 0-7), (next K-step, 8-15).
+      // Even and odd K-steps accumulate separately: two chains of 9 MMAs
+      // instead of one of 18.
       const uint32_t rowaddr = st + (8 * nt + (lane & 7)) * kRowStride + ((lane >> 3) & 1) * 16 + (lane >> 4) * 32;
+      float d1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kk = 0; kk < kHalfK; kk += 2) {
         const int ks = kh * kHalfK + kk;
         uint32_t bq[4];
         ldsm_x4(bq, rowaddr + ks * 32);
         mma_bf16(d, qfrag[ks * 32 + lane], bq[0], bq[1]);
-        mma_bf16(d, qfrag[(ks + 1) * 32 + lane], bq[2], bq[3]);
+        mma_bf16(d1, qfrag[(ks + 1) * 32 + lane], bq[2], bq[3]);
       }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) d[c] += d1[c];
     }
     if (kh == 1) spart[nt * 32 + lane] = make_float4(d[0], d[1], d[2], d[3]);
     named_barrier();
@@ -309,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
     }
     named_barrier();
     // every warp is past the output MMAs of stage k-1, the last reader of its ring slot
-    if (warp == 0) issue_stage(k + kNS - 1);
+    if (warp == 0) issue_stage(k + kNS - 1, next_page);
 
     // ---- output: O[16 rows, channels 64 warp .. +63] += P_hi.C + P_lo.C ----
     {
