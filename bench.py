@@ -608,16 +608,16 @@ def main():
     h2d = (h_qc.numel() + h_qr.numel() + h_nc.numel() + h_nr.numel()) * 2
     d2h = h_outs[0].numel() * 2 + h_lses[0].numel() * 4
 
-    # the small-row kernel (s_q*H <= 16) fuses the append for INT4/INT4 g64 only
-    fused = (w.s_q * w.H > 16) or (w.bits_c, w.group_c, w.bits_r, w.group_r) == (4, 64, 4, 64)
-    # the tensor-core path plans a multi-wave split grid with one more (single-block)
-    # kernel: its work list, units longest first (the library's rule, restated here)
+    # a step is one decode launch (the append runs inside the tensor-core and the small-row
+    # kernels), the combine for split plans, and, on the tensor-core path, one more
+    # (single-block) kernel for a multi-wave split grid: its work list, units longest first
+    # (the library's rule, restated here)
     rows = w.s_q * w.H
     units = w.B * n_split * ((rows + 127) // 128)
     chunk_pages = -(-((max_len + 63) // 64) // n_split)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     planned = rows > 16 and n_split > 1 and chunk_pages <= 128 and units > 2 * (sms // 2)
-    launches_per_step = (1 if fused else 2) + (1 if n_split > 1 else 0) + (1 if planned else 0)
+    launches_per_step = 1 + (1 if n_split > 1 else 0) + (1 if planned else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",

@@ -1,28 +1,31 @@
 // Decode for few query rows (s_q * H <= 16) on warp-level tensor-core MMAs
 // (mma.sync m16n8k16). With 16 rows a 128-row tcgen05 tile would be 7/8
 // padding, so this kernel keeps the rows at the MMA's native M = 16 and lets
-// the tokens carry the N and K dimensions.
+// the tokens carry the N and K dimensions. Every cache format: INT4 or INT2
+// codes, groups of 32 or 64 channels, for the content and the RoPE part.
 //
 // Absorbed MQA decode over the low-bit latent cache: scores
 // (q_c . c_hat_t + q_r . kr_hat_t) * scale, softmax, output sum_t p_t c_hat_t
 // (Group-Query Latent Attention abstract: one absorbed decoding path over the
 // shared latent; QuantMLA abstract: dequantization inside the attention).
 //
-// Scores are exact in the codes. For a 64-channel group with scale s and
-// zero z, q . c_hat = s * (q . (u + 128)) + (z - 128 s) * sum(q): the MMA takes
-// the integer codes as bf16 values u + 128 (exact, built by a byte permute),
-// q is bf16, products are exact and accumulate in fp32; s and z are applied
-// per (token, group) in fp32 afterwards. The output is exact in the codes as
-// well: for a group, sum_t p_t c_hat_t = sum_t (p_t s_t) u_t + sum_t p_t z_t.
-// The MMA takes the codes as the exact fp16 values u * 2^-24 (the subnormal
-// whose bits are [u, 0x00]) and the weights w_t = p_t s_t as an fp16 hi + lo
-// pair (22 significant bits, two MMAs); the epilogue scales by 2^24 and adds
-// sum_t p_t z_t, accumulated in fp32 per (row, group).
+// Scores are exact in the codes. For a group with scale s and zero z,
+// q . c_hat = s * (q . (u + 128)) + (z - 128 s) * sum(q): the MMA takes the
+// integer codes as bf16 values u + 128 (exact, built by byte permutes), q is
+// bf16, products are exact and accumulate in fp32; s and z are applied per
+// (token, group) in fp32 afterwards, so every group has its own MMA chain. The
+// output is exact in the codes as well: for a group, sum_t p_t c_hat_t =
+// sum_t (p_t s_t) u_t + sum_t p_t z_t. The MMA takes the codes as the exact
+// fp16 values u * 2^-24 (the subnormal whose bits are [u, 0x00]) and the
+// weights w_t = p_t s_t as an fp16 hi + lo pair (22 significant bits, two
+// MMAs); the epilogue scales by 2^24 and adds sum_t p_t z_t, accumulated in
+// fp32 per (row, group). An output N-tile of 8 channels lies in one group, so
+// one weight operand serves it.
 //
 // One CTA per (request, split): whole 64-token pages are bulk-copied into a
 // 4-stage ring (issued by one thread, three pages ahead); eight warps split each page's tokens for
-// the scores (8 keys each) and its channels for the output (one 64-channel
-// group each, the accumulators stay in registers). One named barrier per page hands the
+// the scores (8 keys each) and its channels for the output (64 channels each,
+// the accumulators stay in registers). One named barrier per page hands the
 // weights and per-warp maxima across; the running maximum is lazy (it moves
 // only when a score exceeds it by more than 2^8), so the common page needs no
 // rescale.
@@ -42,7 +45,7 @@ constexpr int kWarps = 8;                    // compute warps
 constexpr int kThreads = 32 * kWarps;
 constexpr int kNS = 4;                       // page stages
 constexpr int kRows = 16;                    // MMA M
-constexpr int kGroups = 9;                   // 8 content groups of 64 + the RoPE group of 64
+constexpr int kKSteps = kDqk / 16;           // 36 score K-steps: the content groups', then the RoPE groups'
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr unsigned kFull = 0xffffffffu;
@@ -53,12 +56,13 @@ constexpr float kCodeScale = 16777216.0f;    // 2^24: the output MMA sees the co
 
 template <class G>
 struct Layout {
+  static constexpr int kGroups = G::kGroupsC + G::kGroupsR;   // scale groups of a token
   static constexpr int kStage = (G::kPageBytes + 127) / 128 * 128;
-  static constexpr int kOffQ = kNS * kStage;                  // Q A-fragments [group][k-step][lane] x 16 B
-  static constexpr int kOffQSum = kOffQ + kGroups * 4 * 32 * 16;  // [group][row] float
+  static constexpr int kOffQ = kNS * kStage;                  // Q A-fragments [K-step][lane] x 16 B
+  static constexpr int kOffQSum = kOffQ + kKSteps * 32 * 16;  // [group][row] float
   static constexpr int kOffP = kOffQSum + kGroups * kRows * 4;    // [2][16 rows][kPRow] fp32 weights
-  static constexpr int kOffM = kOffP + 2 * kPTile;                // [2][16 rows][4 warps] float maxima
-  static constexpr int kOffL = kOffM + 2 * kRows * kWarps * 4;    // [16 rows][4 warps] float row sums
+  static constexpr int kOffM = kOffP + 2 * kPTile;                // [2][16 rows][8 warps] float maxima
+  static constexpr int kOffL = kOffM + 2 * kRows * kWarps * 4;    // [16 rows][8 warps] float row sums
   static constexpr int kOffBar = kOffL + kRows * kWarps * 4;      // full[kNS]
   static constexpr int kOffMisc = kOffBar + kNS * 8;              // abort flag, stage page ids
   static constexpr int kBytes = kOffMisc + 64;
@@ -73,16 +77,16 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // Byte j of a -> byte 0, byte j of b -> byte 2; bytes 1 and 3 replicate the
-// sign bit of those bytes, which is 0 for the nibble-per-byte inputs used here.
+// sign bit of those bytes, which is 0 for the small code values used here.
 __host__ __device__ constexpr uint32_t sel_pair(int j) {
   return static_cast<uint32_t>(j | ((8 | j) << 4) | ((4 + j) << 8) | ((12 + j) << 12));
 }
 
-// Four 16-bit operand pairs from two nibble-per-byte words a, b (values
-// 0..15 in the low half of each byte): pair j = (a.byte j, b.byte j), each
-// completed with the high byte hb (0x43: bf16 128 + u; 0x64: fp16 1024 + u).
-// Three byte permutes per two pairs: interleave first, then merge the constant.
-__device__ __forceinline__ void nibble_pairs(uint32_t a, uint32_t b, uint32_t hb4, uint32_t (&p)[4]) {
+// Four 16-bit operand pairs from two words a, b of one small code per byte
+// (values 0..15): pair j = (a.byte j, b.byte j), each completed with the high
+// byte hb (0x43: bf16 128 + u). Three byte permutes per two pairs: interleave
+// first, then merge the constant.
+__device__ __forceinline__ void byte_pairs(uint32_t a, uint32_t b, uint32_t hb4, uint32_t (&p)[4]) {
   const uint32_t m01 = prmt(a, b, 0x5140u), m23 = prmt(a, b, 0x7362u);  // [a0 b0 a1 b1], [a2 b2 a3 b3]
   p[0] = prmt(m01, hb4, 0x4140u);  // [a0, hb, b0, hb]
   p[1] = prmt(m01, hb4, 0x4342u);  // [a1, hb, b1, hb]
@@ -90,7 +94,7 @@ __device__ __forceinline__ void nibble_pairs(uint32_t a, uint32_t b, uint32_t hb
   p[3] = prmt(m23, hb4, 0x4342u);
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_bf16_frag(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -119,11 +123,106 @@ __device__ __forceinline__ void split_h2(float x0, float x1, uint32_t& hi, uint3
   lo = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
 }
 
+// Score B fragments of one group for this lane: the lane's GS/4 contiguous
+// channels of its key (GS * BITS / 32 bytes at p), K-step s taking channels
+// 4s + {0, 1} (b[s][0]) and 4s + {2, 3} (b[s][1]) as bf16 128 + u.
+template <int BITS, int GS>
+__device__ __forceinline__ void qk_codes(const uint8_t* p, uint32_t (&bf)[GS / 16][2]) {
+  constexpr uint32_t kHB = 0x43434343u;
+  if constexpr (BITS == 4) {
+    // byte i holds channels 2i (low nibble) and 2i + 1: K-step s uses bytes 2s, 2s + 1
+    uint32_t cw[GS / 32];
+    if constexpr (GS == 64) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      cw[0] = v.x;
+      cw[1] = v.y;
+    } else {
+      cw[0] = *reinterpret_cast<const uint32_t*>(p);
+    }
+#pragma unroll
+    for (int i = 0; i < GS / 32; ++i) {
+      uint32_t q[4];
+      byte_pairs(cw[i] & 0x0F0F0F0Fu, (cw[i] >> 4) & 0x0F0F0F0Fu, kHB, q);
+      bf[2 * i][0] = q[0];
+      bf[2 * i][1] = q[1];
+      bf[2 * i + 1][0] = q[2];
+      bf[2 * i + 1][1] = q[3];
+    }
+  } else {
+    // byte s holds channels 4s .. 4s + 3 in bits 0-1, 2-3, 4-5, 6-7
+    const uint32_t cw = GS == 64 ? *reinterpret_cast<const uint32_t*>(p)
+                                 : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p));
+    uint32_t p01[4], p23[4];
+    byte_pairs(cw & 0x03030303u, (cw >> 2) & 0x03030303u, kHB, p01);
+    byte_pairs((cw >> 4) & 0x03030303u, (cw >> 6) & 0x03030303u, kHB, p23);
+#pragma unroll
+    for (int st = 0; st < GS / 16; ++st) {
+      bf[st][0] = p01[st];
+      bf[st][1] = p23[st];
+    }
+  }
+}
+
+// Partial scores of one group: (s * D + (z - 128 s) * sum(q)) for this lane's
+// accumulator entries (rows r, r + 8; keys tl0, tl0 + 1) added into sc.
+// codes: the lane's bytes of key 8w + r; qf: the group's first Q fragment of
+// this lane; meta: (s, z) of key tl0 (key tl0 + 1 at + meta_stride); qs: the
+// group's q sums of row r (row r + 8 at + 8).
+template <int BITS, int GS>
+__device__ __forceinline__ void qk_group(const uint8_t* codes, const uint4* qf, const uint8_t* meta, int meta_stride,
+                                         const float* qs, float (&sc)[4]) {
+  uint32_t bq[GS / 16][2];
+  qk_codes<BITS, GS>(codes, bq);
+  float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int ks = 0; ks < GS / 16; ++ks) mma_bf16_frag(d, qf[ks * 32], bq[ks][0], bq[ks][1]);
+  const uint32_t m0 = *reinterpret_cast<const uint32_t*>(meta);
+  const uint32_t m1 = *reinterpret_cast<const uint32_t*>(meta + meta_stride);
+  const float2 sz0 = __half22float2(bits_h2(m0)), sz1 = __half22float2(bits_h2(m1));  // (s, z)
+  const float e0 = fmaf(-128.0f, sz0.x, sz0.y), e1 = fmaf(-128.0f, sz1.x, sz1.y);
+  const float qa = qs[0], qb = qs[8];
+  sc[0] = fmaf(sz0.x, d[0], fmaf(e0, qa, sc[0]));
+  sc[1] = fmaf(sz1.x, d[1], fmaf(e1, qa, sc[1]));
+  sc[2] = fmaf(sz0.x, d[2], fmaf(e0, qb, sc[2]));
+  sc[3] = fmaf(sz1.x, d[3], fmaf(e1, qb, sc[3]));
+}
+
+// Spread the eight 2-bit fields of x (bits 2j, 2j + 1) to nibbles (bits 4j, 4j + 1).
+__device__ __forceinline__ uint32_t spread_crumbs(uint32_t x) {
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  return (x | (x << 2)) & 0x33333333u;
+}
+
+// Output codes of one key for lane column n of the warp's 64 channels (content
+// codes of the key at p): nibble j is the code of output N-tile j's column n.
+// Groups of 64: tile j column n is channel 8n + j; groups of 32: tiles 0-3
+// take the first group (channel 4n + j), tiles 4-7 the second (4n + j - 4).
+template <int BITS, int GS>
+__device__ __forceinline__ uint32_t pv_codes(const uint8_t* p, int n) {
+  if constexpr (BITS == 4 && GS == 64) {
+    return *reinterpret_cast<const uint32_t*>(p + 4 * n);
+  } else if constexpr (BITS == 4) {
+    return static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p + 2 * n)) |
+           (static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p + 16 + 2 * n)) << 16);
+  } else if constexpr (GS == 64) {
+    return spread_crumbs(*reinterpret_cast<const uint16_t*>(p + 2 * n));
+  } else {
+    return spread_crumbs(static_cast<uint32_t>(p[n]) | (static_cast<uint32_t>(p[8 + n]) << 8));
+  }
+}
+
+// Channel (of the warp's 64) of output N-tile j, column n.
+template <int GS>
+__device__ __forceinline__ int pv_channel(int j, int n) {
+  return GS == 64 ? 8 * n + j : 32 * (j >> 2) + 4 * n + (j & 3);
+}
+
 template <int BITS_C, int G_C, int BITS_R, int G_R>
 __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeArgs a) {
   using G = QGeom<BITS_C, G_C, BITS_R, G_R>;
   using Lo = Layout<G>;
-  static_assert(BITS_C == 4 && G_C == 64 && BITS_R == 4 && G_R == 64, "INT4 g64 content and RoPE");
+  static_assert(Lo::kGroups * kRows <= 2 * kThreads, "q sums: at most two (group, row) entries per thread");
   // launched as a programmatic dependent: wait for the previous grid before any read
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
@@ -209,74 +308,89 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
     const int lim0 = row_ok0 ? min(row_visible(T, a.s_q, a.H, r), t_end) : 0;
     const int lim1 = row_ok1 ? min(row_visible(T, a.s_q, a.H, r + 8), t_end) : 0;
 
-    // Q as A fragments, one 16-byte entry per (group, k-step, lane). Within a
-    // 64-channel group, K-step s pairs logical columns {2kp, 2kp+1} with
-    // channels 16kp + 4s + {0,1} and {8+2kp, 9+2kp} with 16kp + 4s + {2,3}:
-    // the code bytes one lane needs for all four K-steps are then the 8
-    // contiguous bytes [8kp, 8kp+8) of the token's group.
+    // Q as A fragments, one 16-byte entry per (K-step, lane); the K-steps run
+    // over the content groups, then the RoPE groups, GS/16 per group of GS
+    // channels. Within a group, K-step s pairs logical columns {2kp, 2kp+1}
+    // with channels (GS/4) kp + 4s + {0,1} and {8+2kp, 9+2kp} with
+    // (GS/4) kp + 4s + {2,3}: the code bytes one lane needs for all of the
+    // group's K-steps are then contiguous in the token's group.
     {
       const uint32_t* qc = reinterpret_cast<const uint32_t*>(a.q_c);
       const uint32_t* qr = reinterpret_cast<const uint32_t*>(a.q_r);
       uint4* qf = reinterpret_cast<uint4*>(smem + Lo::kOffQ);
       // Every load of the set-up is issued before the first use of any, so
       // the set-up costs one round trip to memory (it precedes the first page).
-      constexpr int kEntries = kGroups * 4 * 32;
+      constexpr int kEntries = kKSteps * 32;
       constexpr int kPerThread = (kEntries + kWarps * 32 - 1) / (kWarps * 32);
+      constexpr int kStepsC = kDc / 16;  // content K-steps
       uint4 fv[kPerThread];
 #pragma unroll
       for (int k = 0; k < kPerThread; ++k) {
         const int e = tid + k * kWarps * 32;
         fv[k] = make_uint4(0, 0, 0, 0);
         if (e < kEntries) {
-          const int g = e / 128, s = (e / 32) & 3, ln = e & 31;
+          const int ks = e / 32, ln = e & 31;
           const int er = ln >> 2, ekp = ln & 3;
-          const int c = 16 * ekp + 4 * s;  // channel within the group
+          const bool rope = ks >= kStepsC;
+          const int gs = rope ? G_R : G_C, kr = rope ? ks - kStepsC : ks;
+          const int g = kr / (gs / 16), st = kr % (gs / 16);
+          const int c = g * gs + (gs / 4) * ekp + 4 * st;  // channel within q_c or q_r
           const bool ok0 = er < a.rows, ok1 = er + 8 < a.rows;
           const size_t q0 = static_cast<size_t>(b) * a.rows + er, q1 = q0 + 8;
           auto ld = [&](bool ok, size_t q, int cc) -> uint32_t {
             if (!ok) return 0u;
-            return g < 8 ? __ldg(qc + (q * kDc + 64 * g + cc) / 2) : __ldg(qr + (q * kDr + cc) / 2);
+            return rope ? __ldg(qr + (q * kDr + cc) / 2) : __ldg(qc + (q * kDc + cc) / 2);
           };
           fv[k] = make_uint4(ld(ok0, q0, c), ld(ok1, q1, c), ld(ok0, q0, c + 2), ld(ok1, q1, c + 2));
         }
       }
       // per (group, row) sums of q, for the zero-point and code-offset term:
-      // a group's 64 channels as eight 16-byte loads
-      const int eg = tid / kRows, erow = tid % kRows;  // threads 0..143: (group, row)
-      const bool sum_ok = tid < kGroups * kRows && erow < a.rows;
-      uint4 qv[8];
-      if (sum_ok) {
-        const uint4* q = reinterpret_cast<const uint4*>(
-            (eg < 8) ? a.q_c + (static_cast<size_t>(b) * a.rows + erow) * kDc + 64 * eg
-                     : a.q_r + (static_cast<size_t>(b) * a.rows + erow) * kDr);
+      // a group's channels as 16-byte loads, at most two entries per thread
+      constexpr int kSumEntries = Lo::kGroups * kRows;
+      constexpr int kSumPer = (kSumEntries + kThreads - 1) / kThreads;
+      constexpr int kMaxV = (G_C > G_R ? G_C : G_R) / 8;
+      uint4 qv[kSumPer][kMaxV];
 #pragma unroll
-        for (int v = 0; v < 8; ++v) qv[v] = __ldg(q + v);
+      for (int i = 0; i < kSumPer; ++i) {
+        const int e = tid + i * kThreads;
+        const int eg = e / kRows, erow = e % kRows;
+        const bool ok = e < kSumEntries && erow < a.rows;
+        const bool rope = eg >= G::kGroupsC;
+        const int nv = (rope ? G_R : G_C) / 8;
+        const uint4* q = reinterpret_cast<const uint4*>(
+            rope ? a.q_r + (static_cast<size_t>(b) * a.rows + erow) * kDr + G_R * (eg - G::kGroupsC)
+                 : a.q_c + (static_cast<size_t>(b) * a.rows + erow) * kDc + G_C * eg);
+#pragma unroll
+        for (int v = 0; v < kMaxV; ++v) qv[i][v] = (ok && v < nv) ? __ldg(q + v) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int k = 0; k < kPerThread; ++k)
         if (tid + k * kWarps * 32 < kEntries) qf[tid + k * kWarps * 32] = fv[k];
-      if (tid < kGroups * kRows) {
-        float acc = 0.0f;
-        if (sum_ok) {
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint32_t wv[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
+      for (int i = 0; i < kSumPer; ++i) {
+        const int e = tid + i * kThreads;
+        if (e < kSumEntries) {
+          float acc = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc += bf16_lo(wv[e]) + bf16_hi(wv[e]);
+          for (int v = 0; v < kMaxV; ++v) {
+            const uint32_t wv[4] = {qv[i][v].x, qv[i][v].y, qv[i][v].z, qv[i][v].w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) acc += bf16_lo(wv[x]) + bf16_hi(wv[x]);
           }
+          reinterpret_cast<float*>(smem + Lo::kOffQSum)[e] = acc;  // [group][row]
         }
-        reinterpret_cast<float*>(smem + Lo::kOffQSum)[tid] = acc;  // [group][row]
       }
       named_barrier_compute();
     }
     const uint4* qfrag = reinterpret_cast<const uint4*>(smem + Lo::kOffQ);
     const float* qsum = reinterpret_cast<const float*>(smem + Lo::kOffQSum);
-    float o[8][4];  // output accumulators of group w: block j, fragment c (see the epilogue)
+    constexpr int kPvGroups = 64 / G_C;  // scale groups among a warp's 64 output channels
+    float o[8][4];  // output accumulators of channels 64w .. 64w+63: N-tile j, fragment c (see the epilogue)
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
     float m_run[2] = {-CUDART_INF_F, -CUDART_INF_F};  // running maximum (log2 units) of rows r, r+8
     float l_acc[2] = {0.0f, 0.0f};                      // this thread's share of the row sums, scaled to m_run
-    float corr[2] = {0.0f, 0.0f};                       // this thread's share of sum p z of group w, rows r, r+8
+    float corr[kPvGroups][2] = {};                      // this thread's share of sum p z per group, rows r, r+8
     const float sl2 = a.scale_log2;
 
     for (int k = 0; k < n_pages; ++k) {
@@ -299,32 +413,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
       const int tlb = 8 * w + r;       // key of this lane's B column
       const int tl0 = 8 * w + 2 * kp;  // keys of this lane's accumulator columns: tl0, tl0 + 1
 #pragma unroll
-      for (int g = 0; g < kGroups; ++g) {
-        const uint2 cw = *reinterpret_cast<const uint2*>(
-            st + (g < 8 ? G::kOffCC + tlb * G::kRowC + 32 * g : G::kOffRC + tlb * G::kRowR) + 8 * kp);
-        // code byte i of the lane's 8 -> bf16 pair (128 + u_even, 128 + u_odd); K-step ks uses bytes 2ks, 2ks+1
-        uint32_t bq[2][4];
-        nibble_pairs(cw.x & 0x0F0F0F0Fu, (cw.x >> 4) & 0x0F0F0F0Fu, 0x43434343u, bq[0]);
-        nibble_pairs(cw.y & 0x0F0F0F0Fu, (cw.y >> 4) & 0x0F0F0F0Fu, 0x43434343u, bq[1]);
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int g = 0; g < G::kGroupsC; ++g)
+        qk_group<BITS_C, G_C>(st + G::kOffCC + tlb * G::kRowC + g * (G_C * BITS_C / 8) + kp * (G_C * BITS_C / 32),
+                              qfrag + g * (G_C / 16) * 32 + lane, st + G::kOffCM + tl0 * G::kGroupsC * 4 + 4 * g,
+                              G::kGroupsC * 4, qsum + g * kRows + r, sc);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint4 af = qfrag[(g * 4 + ks) * 32 + lane];
-          mma_bf16(d, af, bq[ks >> 1][2 * (ks & 1)], bq[ks >> 1][2 * (ks & 1) + 1]);
-        }
-        // s * D + (z - 128 s) * sum(q) for this lane's two keys
-        const uint32_t m0 = *reinterpret_cast<const uint32_t*>(
-            st + (g < 8 ? G::kOffCM + tl0 * G::kGroupsC * 4 + 4 * g : G::kOffRM + tl0 * 4));
-        const uint32_t m1 = *reinterpret_cast<const uint32_t*>(
-            st + (g < 8 ? G::kOffCM + (tl0 + 1) * G::kGroupsC * 4 + 4 * g : G::kOffRM + (tl0 + 1) * 4));
-        const float2 sz0 = __half22float2(bits_h2(m0)), sz1 = __half22float2(bits_h2(m1));  // (s, z)
-        const float e0 = fmaf(-128.0f, sz0.x, sz0.y), e1 = fmaf(-128.0f, sz1.x, sz1.y);
-        const float qa = qsum[g * kRows + r], qb = qsum[g * kRows + r + 8];
-        sc[0] = fmaf(sz0.x, d[0], fmaf(e0, qa, sc[0]));
-        sc[1] = fmaf(sz1.x, d[1], fmaf(e1, qa, sc[1]));
-        sc[2] = fmaf(sz0.x, d[2], fmaf(e0, qb, sc[2]));
-        sc[3] = fmaf(sz1.x, d[3], fmaf(e1, qb, sc[3]));
-      }
+      for (int g = 0; g < G::kGroupsR; ++g)
+        qk_group<BITS_R, G_R>(st + G::kOffRC + tlb * G::kRowR + g * (G_R * BITS_R / 8) + kp * (G_R * BITS_R / 32),
+                              qfrag + (kDc / 16 + g * (G_R / 16)) * 32 + lane,
+                              st + G::kOffRM + tl0 * G::kGroupsR * 4 + 4 * g, G::kGroupsR * 4,
+                              qsum + (G::kGroupsC + g) * kRows + r, sc);
 
       // ---- masks, this warp's maximum, weights ----
       float mloc[2] = {-CUDART_INF_F, -CUDART_INF_F};
@@ -382,7 +480,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
         alpha[i] = (mnew[i] == -CUDART_INF_F) ? 1.0f : exp2f(m_run[i] - mnew[i]);
         const float own = (mw[i] == -CUDART_INF_F) ? 0.0f : exp2f(mw[i] - mnew[i]);
         l_acc[i] = l_acc[i] * alpha[i] + l_own[i] * own;
-        corr[i] *= alpha[i];
+#pragma unroll
+        for (int pg = 0; pg < kPvGroups; ++pg) corr[pg][i] *= alpha[i];
         m_run[i] = mnew[i];
       }
       if (__any_sync(kFull, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
@@ -396,11 +495,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
       }
       const bool rescale_w = __any_sync(kFull, !uniform);
 
-      // ---- O[16 rows, group w] += sum_t p_t c_hat_t over the page ----
-      // Block j, column n holds channel 64w + 8n + j: lane (r, kp) supplies
-      // column r from code word r of the group's 32 bytes. K-step ks takes keys
-      // 16ks + [0, 16), scored by warps 2ks and 2ks+1; their weights were taken
-      // against those warps' maxima and are scaled to the new one.
+      // ---- O[16 rows, channels 64w .. 64w+63] += sum_t p_t c_hat_t over the page ----
+      // Lane (r, kp) supplies column r of every N-tile (pv_codes and
+      // pv_channel give the channels); an N-tile lies in one scale group. K-step
+      // ks takes keys 16ks + [0, 16), scored by warps 2ks and 2ks+1; their
+      // weights were taken against those warps' maxima and are scaled to the
+      // new one.
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         const int ta = 16 * ks + 2 * kp, tb = ta + 8;  // page-local keys of B rows {0,1} and {8,9}
@@ -422,42 +522,53 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
             pw[q].y *= fq[q];
           }
         }
-        // (s, z) of group w for keys ta, ta+1, tb, tb+1; keys past the end (or
-        // of a missing page) get s = z = 0, so garbage never reaches the MMA
-        float sv[4], zv[4];
+        // (s, z) of the warp's groups for keys ta, ta+1, tb, tb+1; keys past
+        // the end (or of a missing page) get s = z = 0, so garbage never
+        // reaches the MMA
+        float sv[kPvGroups][4], zv[kPvGroups][4];
         uint32_t wd[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int t = (q < 2 ? ta : tb) + (q & 1);
           const bool ok = page_ok && P0 + t < t_end;
-          const uint32_t m = ok ? *reinterpret_cast<const uint32_t*>(st + G::kOffCM + t * G::kGroupsC * 4 + 4 * w) : 0u;
-          const float2 sz = __half22float2(bits_h2(m));
-          sv[q] = sz.x;
-          zv[q] = sz.y;
-          wd[q] = *reinterpret_cast<const uint32_t*>(st + G::kOffCC + t * G::kRowC + 32 * w + 4 * r);
+#pragma unroll
+          for (int pg = 0; pg < kPvGroups; ++pg) {
+            const uint32_t m =
+                ok ? *reinterpret_cast<const uint32_t*>(st + G::kOffCM + t * G::kGroupsC * 4 + 4 * (kPvGroups * w + pg))
+                   : 0u;
+            const float2 sz = __half22float2(bits_h2(m));
+            sv[pg][q] = sz.x;
+            zv[pg][q] = sz.y;
+          }
+          wd[q] = pv_codes<BITS_C, G_C>(st + G::kOffCC + t * G::kRowC + 8 * BITS_C * w, r);
         }
         // A = w = p * s as fp16 hi + lo; the zero-point term sum p z in fp32
-        uint32_t ah[4], al[4];
+        uint32_t ah[kPvGroups][4], al[kPvGroups][4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int k0 = (q < 2) ? 0 : 2;  // keys (ta, ta+1) or (tb, tb+1)
-          split_h2(pw[q].x * sv[k0], pw[q].y * sv[k0 + 1], ah[q], al[q]);
-          corr[q & 1] = fmaf(pw[q].x, zv[k0], fmaf(pw[q].y, zv[k0 + 1], corr[q & 1]));
+        for (int pg = 0; pg < kPvGroups; ++pg) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int k0 = (q < 2) ? 0 : 2;  // keys (ta, ta+1) or (tb, tb+1)
+            split_h2(pw[q].x * sv[pg][k0], pw[q].y * sv[pg][k0 + 1], ah[pg][q], al[pg][q]);
+            corr[pg][q & 1] = fmaf(pw[q].x, zv[pg][k0], fmaf(pw[q].y, zv[pg][k0 + 1], corr[pg][q & 1]));
+          }
         }
-        // B: channel j of keys (ta, ta+1) and (tb, tb+1). The 16-bit pattern
-        // [u, 0x00] is the fp16 value u * 2^-24 (subnormal, exact): one byte
-        // permute per pair, no offset to cancel; the epilogue scales by 2^24.
+        // B: code nibble j of keys (ta, ta+1) and (tb, tb+1). The 16-bit
+        // pattern [u, 0x00] is the fp16 value u * 2^-24 (subnormal, exact):
+        // one byte permute per pair, no offset to cancel; the epilogue scales
+        // by 2^24.
         const uint32_t la0 = wd[0] & 0x0F0F0F0Fu, ha0 = (wd[0] >> 4) & 0x0F0F0F0Fu;
         const uint32_t la1 = wd[1] & 0x0F0F0F0Fu, ha1 = (wd[1] >> 4) & 0x0F0F0F0Fu;
         const uint32_t lb0 = wd[2] & 0x0F0F0F0Fu, hb0 = (wd[2] >> 4) & 0x0F0F0F0Fu;
         const uint32_t lb1 = wd[3] & 0x0F0F0F0Fu, hb1 = (wd[3] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
+          const int pg = j / (8 / kPvGroups);
           const uint32_t sel = sel_pair(j >> 1);
           const uint32_t b0 = (j & 1) ? prmt(ha0, ha1, sel) : prmt(la0, la1, sel);
           const uint32_t b1 = (j & 1) ? prmt(hb0, hb1, sel) : prmt(lb0, lb1, sel);
-          mma_f16(o[j], ah, b0, b1);
-          mma_f16(o[j], al, b0, b1);
+          mma_f16(o[j], ah[pg], b0, b1);
+          mma_f16(o[j], al[pg], b0, b1);
         }
       }
     }
@@ -467,8 +578,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
     for (int i = 0; i < 2; ++i) {
       l_acc[i] += __shfl_xor_sync(kFull, l_acc[i], 1);
       l_acc[i] += __shfl_xor_sync(kFull, l_acc[i], 2);
-      corr[i] += __shfl_xor_sync(kFull, corr[i], 1);  // every lane of the row needs the group's full term
-      corr[i] += __shfl_xor_sync(kFull, corr[i], 2);
+#pragma unroll
+      for (int pg = 0; pg < kPvGroups; ++pg) {  // every lane of the row needs the group's full term
+        corr[pg][i] += __shfl_xor_sync(kFull, corr[pg][i], 1);
+        corr[pg][i] += __shfl_xor_sync(kFull, corr[pg][i], 2);
+      }
     }
     float* lt = reinterpret_cast<float*>(smem + Lo::kOffL);
     if (kp == 0) {
@@ -489,9 +603,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_small_kernel(const DecodeA
     for (int j = 0; j < 8; ++j) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int ch = 64 * w + 8 * (2 * kp + e) + j;
-        otile[r * kORow + ch] = fmaf(o[j][e], kCodeScale, corr[0]) * inv[0];
-        otile[(r + 8) * kORow + ch] = fmaf(o[j][2 + e], kCodeScale, corr[1]) * inv[1];
+        const int ch = 64 * w + pv_channel<G_C>(j, 2 * kp + e);
+        const int pg = j / (8 / kPvGroups);
+        otile[r * kORow + ch] = fmaf(o[j][e], kCodeScale, corr[pg][0]) * inv[0];
+        otile[(r + 8) * kORow + ch] = fmaf(o[j][2 + e], kCodeScale, corr[pg][1]) * inv[1];
       }
     }
     const size_t part_row0 = (static_cast<size_t>(b) * a.n_split + split) * a.rows;
@@ -559,14 +674,27 @@ cudaError_t launch_t(const DecodeLaunch& L) {
 }  // namespace small
 
 bool decode_small_supported(const DecodeLaunch& L) {
-  return L.quantized && L.s_q * L.H <= small::kRows && L.num_pages >= 1 && L.bits_c == 4 && L.group_c == 64 &&
-         L.bits_r == 4 && L.group_r == 64;
+  auto bits_ok = [](int bits) { return bits == 2 || bits == 4; };
+  auto group_ok = [](int g) { return g == 32 || g == 64; };
+  return L.quantized && L.s_q * L.H <= small::kRows && L.num_pages >= 1 && bits_ok(L.bits_c) && bits_ok(L.bits_r) &&
+         group_ok(L.group_c) && group_ok(L.group_r);
 }
 
 cudaError_t launch_decode_small(const DecodeLaunch& L) {
   if (!L.quantized) return launch_decode_small_bf16(L);
   if (!decode_small_supported(L)) return cudaErrorNotSupported;
-  return small::launch_t<4, 64, 4, 64>(L);
+#define MLA_SMALL_CASE(BC, GC, BR, GR)                                            \
+  if (L.bits_c == BC && L.group_c == GC && L.bits_r == BR && L.group_r == GR)   \
+    return small::launch_t<BC, GC, BR, GR>(L);
+#define MLA_SMALL_R(BC, GC) \
+  MLA_SMALL_CASE(BC, GC, 4, 64) MLA_SMALL_CASE(BC, GC, 4, 32) MLA_SMALL_CASE(BC, GC, 2, 64) MLA_SMALL_CASE(BC, GC, 2, 32)
+  MLA_SMALL_R(4, 64)
+  MLA_SMALL_R(4, 32)
+  MLA_SMALL_R(2, 64)
+  MLA_SMALL_R(2, 32)
+#undef MLA_SMALL_R
+#undef MLA_SMALL_CASE
+  return cudaErrorNotSupported;
 }
 
 }  // namespace mla

@@ -221,9 +221,8 @@ mla_status mla_qdecode(const mla_qcache_desc* desc, const void* pool,
  * tokens inside its key range into the pool, then copies its pages in), which
  * saves the append launch and its latency. Results and pool bytes are those of
  * mla_qcache_append (seq_lens_before = seq_lens - n_new) followed by
- * mla_qdecode; where the fused form does not apply (MLA_DECODE_FORCE_SIMT, or
- * a small-row shape in a format the small-row kernel lacks) the library
- * launches the append kernel and then the decode itself.
+ * mla_qdecode; where the fused form does not apply (MLA_DECODE_FORCE_SIMT)
+ * the library launches the append kernel and then the decode itself.
  * (QuantMLA abstract: tokens are quantized as they are written; the
  * workload's verify step appends s_q tokens per request before the decode.)
  *   seq_lens      device int32 [B]: lengths AFTER the append; the new tokens

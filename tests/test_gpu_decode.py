@@ -48,11 +48,18 @@ SMALL = [
     (4, 32, 2, 64, 32, 2, [100, 129]),
     (2, 64, 2, 32, 64, 1, [640, 64]),
     (4, 64, 4, 64, 8, 3, [3, 70]),
-    # at most 16 query rows: the warp-level MMA kernel (INT4 g64)
+    # at most 16 query rows: the warp-level MMA kernel, every format
     (4, 64, 4, 64, 16, 1, [1, 63, 64, 65, 200, 1000]),
     (4, 64, 4, 64, 8, 2, [2, 65, 300, 4096]),
     (4, 64, 4, 64, 5, 3, [100, 1, 129]),
     (4, 64, 4, 64, 1, 1, [33, 640]),
+    (2, 32, 4, 64, 16, 1, [1, 65, 1000]),
+    (2, 32, 4, 64, 8, 2, [2, 130, 777]),
+    (4, 32, 2, 64, 16, 1, [100, 129]),
+    (2, 64, 2, 32, 5, 3, [640, 64, 3]),
+    (4, 32, 4, 32, 16, 1, [300, 63]),
+    (2, 32, 2, 32, 16, 1, [64, 1, 500]),
+    (2, 64, 4, 64, 3, 1, [257]),
 ]
 
 

@@ -21,7 +21,8 @@ CASES = [
     (4, 64, 4, 64, 64, 3, 3, [5, 200], 1, 0),                       # 192 rows: two row tiles both write
     (4, 64, 4, 64, 16, 1, 1, [1024, 7], 0, 0),                      # s_q*H <= 16: fused into the small-row kernel
     (4, 64, 4, 64, 8, 2, 2, [64, 65, 700], 3, 0),                   # small-row kernel, tokens straddle a page edge
-    (2, 32, 4, 64, 16, 1, 1, [300, 9], 0, 0),                       # s_q*H <= 16, INT2: append kernel, then decode
+    (2, 32, 4, 64, 16, 1, 1, [300, 9], 0, 0),                       # s_q*H <= 16, INT2 g32: fused into the small-row kernel
+    (2, 64, 2, 32, 8, 2, 2, [64, 65, 129], 2, 0),                   # small-row kernel, INT2 RoPE, page edge
     (4, 64, 4, 64, 128, 1, 2, [90, 3], 2, MLA_DECODE_FORCE_SIMT),   # SIMT path: append kernel, then decode
 ]
 
