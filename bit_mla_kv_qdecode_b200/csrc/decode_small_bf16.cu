@@ -13,9 +13,11 @@
 // significant bits) and the output takes two terms, P_hi.C + P_lo.C. All
 // accumulation is fp32.
 //
-// One CTA per (request, key split), eight warps, a ring of four stages of 32
-// tokens (half a page). Warp 0 copies a stage's rows with one bulk copy per
-// token into rows padded to 1,168 bytes, so the eight 16-byte row pieces one
+// One CTA per (request, key split), eight warps, two CTAs per SM (the phases
+// of a stage are short and separated by barriers: the other CTA fills the
+// gaps), a ring of two stages of 32 tokens (half a page) per CTA. Warp 4
+// copies the next stage's rows as soon as the current stage's scores are in,
+// with one bulk copy per token into rows padded to 1,168 bytes, so the eight 16-byte row pieces one
 // ldmatrix phase reads fall in distinct banks. Per stage: warp w scores key
 // tile w & 3 (8 keys) over channel half w >> 2 (18 K-steps); warps 4-7 hand
 // their partial sums to warps 0-3 through shared memory, which finish the
@@ -37,7 +39,8 @@ constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
 constexpr int kRows = 16;                    // MMA M
 constexpr int kTok = 32;                     // tokens per stage (half a page)
-constexpr int kNS = 4;                       // stages
+constexpr int kNS = 2;                       // stages (two CTAs per SM: four stages in flight per SM)
+constexpr int kIssueWarp = 4;                // a warp that idles between the score and maximum barriers
 constexpr int kRowBytes = kDqk * 2;          // one token's 576 bf16
 constexpr int kRowStride = kRowBytes + 16;   // 1,168: 292 words, 4 (mod 32) banks apart
 constexpr int kStage = kTok * kRowStride;
@@ -95,7 +98,7 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
   lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) decode_small_bf16_kernel(const DecodeArgs a) {
   // launched as a programmatic dependent: wait for the previous grid before any read
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
@@ -123,8 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
   }
   __syncthreads();
 
-  // Stage k holds tokens t_begin + 32k .. +31, half (k & 1) of one page. Warp
-  // 0 issues it: one bulk copy per token into its padded row; rows past the
+  // Stage k holds tokens t_begin + 32k .. +31, half (k & 1) of one page. The
+  // issuing warp copies it: one bulk copy per token into its padded row; rows past the
   // unit's keys, or of a page the table could not name, are zeroed (their
   // weights are 0, and 0 times stale bytes must not meet a NaN). The zeroing
   // stores come before the arrive that opens the stage's phase.
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
   auto page_of = [&](int k) {
     return k < n_st ? lookup_page(a.table, a.max_pages, a.num_pages, b, t_begin + k * kTok) : -1;
   };
-  auto issue_stage = [&](int k, int page) {  // warp 0, all lanes; page: lookup_page of stage k
+  auto issue_stage = [&](int k, int page) {  // the issuing warp, all lanes; page: lookup_page of stage k
     if (k >= n_st) return;
     const int s = k % kNS;
     const int t0 = t_begin + k * kTok;
@@ -159,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
                      kRowBytes, &full[s]);
     n_issued = k + 1;
   };
-  if (warp == 0)
-    for (int k = 0; k < kNS - 1; ++k) issue_stage(k, page_of(k));
+  if (warp == kIssueWarp)  // every slot is free at the start
+    for (int k = 0; k < kNS; ++k) issue_stage(k, page_of(k));
 
   const int r = lane >> 2, kp = lane & 3;  // MMA fragment coordinates: row group, k pair
   const bool row_ok0 = r < a.rows, row_ok1 = r + 8 < a.rows;
@@ -212,9 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
 
   for (int k = 0; k < n_st; ++k) {
     const int s = k % kNS;
-    // the page of the stage issued after this stage's weights, loaded now so
-    // that warp 0 does not hold the next barrier up
-    const int next_page = warp == 0 ? page_of(k + kNS - 1) : -1;
+    // the page of the stage issued after this stage's scores, loaded now so
+    // that the issuing warp does not hold the next barrier up
+    const int next_page = (warp == kIssueWarp && k > 0) ? page_of(k + kNS - 1) : -1;
     // on a timeout the loop runs on (every warp keeps the same barrier
     // sequence) with the abort flag set, so later waits return at once
     if (!ptx::mbar_wait(&full[s], (k / kNS) & 1, abort_flag, kWaitLimitNs)) {
@@ -247,6 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
     }
     if (kh == 1) spart[nt * 32 + lane] = make_float4(d[0], d[1], d[2], d[3]);
     named_barrier();
+    // every warp is past the output MMAs of stage k-1, the last reader of the
+    // ring slot of stage k + kNS - 1 (issued at the start for k = 0); the
+    // issuing warp has nothing to do until the next barrier
+    if (warp == kIssueWarp && k > 0) issue_stage(k + kNS - 1, next_page);
     if (kh == 0) {
       const float4 p2 = spart[nt * 32 + lane];
       d[0] += p2.x; d[1] += p2.y; d[2] += p2.z; d[3] += p2.w;
@@ -318,8 +325,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
       l_acc[1] *= alpha[1];
     }
     named_barrier();
-    // every warp is past the output MMAs of stage k-1, the last reader of its ring slot
-    if (warp == 0) issue_stage(k + kNS - 1, next_page);
 
     // ---- output: O[16 rows, channels 64 warp .. +63] += P_hi.C + P_lo.C ----
     {
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_small_bf16_kernel(const De
 
   // ---- teardown: after an abort, let every issued stage copy land before the CTA exits ----
   __syncthreads();
-  if (warp == 0 && lane == 0 && *abort_flag) {
+  if (warp == kIssueWarp && lane == 0 && *abort_flag) {
     for (int k = max(0, n_issued - kNS); k < n_issued; ++k)
       ptx::mbar_wait(&full[k % kNS], (k / kNS) & 1, nullptr, kWaitLimitNs);
   }
