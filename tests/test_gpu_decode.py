@@ -203,6 +203,20 @@ def test_full_size_workloads(idx):
         check(case, out, lse, FULL[idx], quantized=False, bf16_out=True)
 
 
+@pytest.mark.parametrize("fmt", [(2, 32, 4, 64), (4, 32, 2, 32)])
+def test_small_rows_full_length_other_formats(fmt):
+    # The memory-bound shape (16 query rows, 32,768 keys, paged) in formats
+    # other than INT4/INT4 g64, on the small-row kernel with its auto split
+    # plan; four requests, every one checked.
+    bc, gc, br, gr = fmt
+    w = synth.workload(5).scaled(B=4, bits_c=bc, group_c=gc, bits_r=br, group_r=gr)
+    case = mc.make_case(w)
+    pool, table_t = mc.fill_pool(case)
+    out, lse = run_decode(case, pool, table_t, out_dtype=torch.bfloat16)
+    assert api.mla_get_device_status() == 0
+    check(case, out, lse, range(w.B), bf16_out=True)
+
+
 def test_long_request_chunk_cap():
     # 32,768 keys asked for as one split: the library raises the split count so
     # that no accumulator sums more than 8,192 keys, which keeps the error well
