@@ -248,7 +248,6 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
 // warps; large batches take a whole row per warp (fewer, longer warps).
 constexpr int kCombineWarps = 8;
 constexpr int kCombineGroup = 4;  // splits in flight per warp
-constexpr long kCombineSmallRows = 148 * 16;  // output rows below which a row is split over four warps
 template <int kParts>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs a) {
   ptx::griddep_wait();
@@ -392,8 +391,14 @@ cudaError_t launch_decode_simt(const DecodeLaunch& L) {
 cudaError_t launch_combine(const DecodeLaunch& L) {
   const DecodeArgs a = make_decode_args(L);
   const long rows = static_cast<long>(a.B) * a.rows;
-  // fewer rows than 16 whole-row warps for each of 148 SMs: split each row over four warps
-  const bool quarter = rows < kCombineSmallRows;
+  // fewer rows than 16 whole-row warps for each SM: split each row over four warps
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const bool quarter = rows < 16L * sms;
   const long blocks = (rows * (quarter ? 4 : 1) + kCombineWarps - 1) / kCombineWarps;
   if (blocks > 0x7FFFFFFFL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(blocks)), block(32 * kCombineWarps);
