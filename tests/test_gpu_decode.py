@@ -135,6 +135,28 @@ def test_empty_request_and_length_errors():
     assert api.mla_get_device_status() == api._lib.MLA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("quantized", [True, False])
+@pytest.mark.parametrize("H", [16, 128])
+@pytest.mark.parametrize("flags", KERNELS)
+@pytest.mark.parametrize("bad_entry", ["past_pool", "unused"])
+def test_bad_table_entry_is_flagged(quantized, H, flags, bad_entry):
+    # One block-table entry inside request 1's pages names no page of the
+    # pool (past its end, or the -1 of an unused slot). Every kernel path
+    # (small-row and tensor-core, quantized and BF16, and the SIMT kernel)
+    # skips that page without reading it, flags the call in the device status
+    # word, and leaves the other requests exact.
+    w = synth.workload(1).scaled(B=3, H=H)
+    case = mc.make_case(w, lens=[200, 300, 130])
+    pool, table_t = mc.fill_pool(case, quantized=quantized)
+    assert api.mla_get_device_status() == 0
+    bad = table_t.clone()
+    bad[1, 2] = case.num_pages + 7 if bad_entry == "past_pool" else -1
+    out, lse = run_decode(case, pool, bad, flags=flags, quantized=quantized)
+    assert api.mla_get_device_status() == api._lib.MLA_ERR_INVALID_ARG
+    assert api.mla_get_device_status() == 0  # reading clears it
+    check(case, out, lse, [0, 2], quantized=quantized)
+
+
 def test_determinism_and_paging_invariance():
     w = synth.workload(2).scaled(B=3, H=128)
     lens = [333, 1024, 65]
