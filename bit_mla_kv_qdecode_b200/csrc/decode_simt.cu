@@ -242,13 +242,13 @@ __global__ void __launch_bounds__(kThreads) decode_simt_kernel(DecodeArgs a) {
 //
 // A warp merges 512 / kParts channels of one output row: lane l holds the
 // 16-byte pieces 32 q + l (q < 4 / kParts) of its part in every split. The
-// loads of four splits (their lse and their pieces) are issued together and
-// merged online against a running maximum, so a row of up to four splits
+// loads of kGroup splits (their lse and their pieces) are issued together and
+// merged online against a running maximum, so a row of up to kGroup splits
 // costs one round trip to memory. kParts = 4 spreads a small batch over more
-// warps; large batches take a whole row per warp (fewer, longer warps).
+// warps and keeps sixteen splits in flight (one piece each); large batches
+// take a whole row per warp (fewer, longer warps; four splits of four pieces).
 constexpr int kCombineWarps = 8;
-constexpr int kCombineGroup = 4;  // splits in flight per warp
-template <int kParts>
+template <int kParts, int kGroup>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs a) {
   ptx::griddep_wait();
   ptx::griddep_launch_dependents();
@@ -271,11 +271,11 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs 
   float4 acc[kVec];
 #pragma unroll
   for (int q = 0; q < kVec; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < n_b; j += kCombineGroup) {
-    float l[kCombineGroup];
-    float4 v[kCombineGroup][kVec];
+  for (int j = 0; j < n_b; j += kGroup) {
+    float l[kGroup];
+    float4 v[kGroup][kVec];
 #pragma unroll
-    for (int u = 0; u < kCombineGroup; ++u) {
+    for (int u = 0; u < kGroup; ++u) {
       const bool in = j + u < n_b;
       l[u] = in ? lse_p[static_cast<size_t>(j + u) * a.rows] : -CUDART_INF_F;
 #pragma unroll
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs 
     }
     float mg = l[0];
 #pragma unroll
-    for (int u = 1; u < kCombineGroup; ++u) mg = fmaxf(mg, l[u]);
+    for (int u = 1; u < kGroup; ++u) mg = fmaxf(mg, l[u]);
     if (mg == -CUDART_INF_F) continue;  // no split of this group saw a key (same values in every lane)
     if (mg > m) {  // the running maximum moves: rescale what is merged so far
       const float f = (m == -CUDART_INF_F) ? 0.0f : exp2f((m - mg) * kLog2e);
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_kernel(DecodeArgs 
       m = mg;
     }
 #pragma unroll
-    for (int u = 0; u < kCombineGroup; ++u) {
+    for (int u = 0; u < kGroup; ++u) {
       const float w = exp2f((l[u] - m) * kLog2e);  // lse -inf -> 0
       tot += w;
 #pragma unroll
@@ -402,8 +402,8 @@ cudaError_t launch_combine(const DecodeLaunch& L) {
   const long blocks = (rows * (quarter ? 4 : 1) + kCombineWarps - 1) / kCombineWarps;
   if (blocks > 0x7FFFFFFFL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(blocks)), block(32 * kCombineWarps);
-  return quarter ? launch_dependent(combine_kernel<4>, grid, block, 0, L.stream, a)
-                 : launch_dependent(combine_kernel<1>, grid, block, 0, L.stream, a);
+  return quarter ? launch_dependent(combine_kernel<4, 16>, grid, block, 0, L.stream, a)
+                 : launch_dependent(combine_kernel<1, 4>, grid, block, 0, L.stream, a);
 }
 
 }  // namespace mla
